@@ -1,0 +1,251 @@
+"""CPU oracle for MoE expert-parallel dispatch / combine (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product path.  The arithmetic lives
+in ep_oracle.c (plain C, single-threaded); this module only marshals numpy
+arrays.  It imports nothing from the CUDA package.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+OK, INVALID_ARG, BAD_EXPERT_ID, CAPACITY = 0, 1, 2, 3
+QUANT = {"none": 0, "fp8": 1, "int8": 2}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"oracle {what}: status {status}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        p = C.c_void_p
+        i32, i64 = C.c_int32, C.c_int64
+        L.oracle_bf16_to_f32.argtypes = [C.c_uint16]
+        L.oracle_bf16_to_f32.restype = C.c_float
+        L.oracle_f32_to_bf16.argtypes = [C.c_float]
+        L.oracle_f32_to_bf16.restype = C.c_uint16
+        L.oracle_e4m3_to_f64.argtypes = [C.c_uint8]
+        L.oracle_e4m3_to_f64.restype = C.c_double
+        L.oracle_f32_to_e4m3.argtypes = [C.c_float]
+        L.oracle_f32_to_e4m3.restype = C.c_uint8
+        L.oracle_pow2_ceil.argtypes = [C.c_float]
+        L.oracle_pow2_ceil.restype = C.c_float
+        L.oracle_layout.argtypes = [p, i32, i32, i32, i32, p, p, p]
+        L.oracle_layout.restype = C.c_int
+        L.oracle_slots.argtypes = [p, p, i32, i32, i32, i32, i32, i64, p, p, p, p, p, p, p]
+        L.oracle_slots.restype = C.c_int
+        L.oracle_quantize_row.argtypes = [p, i32, i32, i32, i32, p, p]
+        L.oracle_quantize_row.restype = C.c_int
+        L.oracle_dispatch_rows.argtypes = [p, i32, i32, i32, p, i32, i32, i32, p, i64, p, p, i64]
+        L.oracle_dispatch_rows.restype = C.c_int
+        L.oracle_combine_rows.argtypes = [p, i64, i32, i32, i32, p, p, p, i64, p]
+        L.oracle_combine_rows.restype = C.c_int
+        L.oracle_round_tokens.argtypes = [i32, i32, i32, i32, p]
+        L.oracle_round_tokens.restype = i64
+        L.oracle_f32_to_e4m3_n.argtypes = [p, i64, p]
+        L.oracle_f32_to_e4m3_n.restype = None
+        L.oracle_f32_to_bf16_n.argtypes = [p, i64, p]
+        L.oracle_f32_to_bf16_n.restype = None
+        L.oracle_e4m3_to_f64_n.argtypes = [p, i64, p]
+        L.oracle_e4m3_to_f64_n.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------------ numbers
+
+def bf16_to_f32(b: np.ndarray) -> np.ndarray:
+    f = lib().oracle_bf16_to_f32
+    return np.array([f(int(v)) for v in np.asarray(b).ravel()], dtype=np.float32).reshape(np.shape(b))
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    a = _c(x, np.float32)
+    out = np.zeros(a.shape, np.uint16)
+    lib().oracle_f32_to_bf16_n(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def e4m3_to_f64(c: np.ndarray) -> np.ndarray:
+    a = _c(c, np.uint8)
+    out = np.zeros(a.shape, np.float64)
+    lib().oracle_e4m3_to_f64_n(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def f32_to_e4m3(x: np.ndarray) -> np.ndarray:
+    a = _c(x, np.float32)
+    out = np.zeros(a.shape, np.uint8)
+    lib().oracle_f32_to_e4m3_n(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def pow2_ceil(s: float) -> float:
+    return lib().oracle_pow2_ceil(float(s))
+
+
+# ------------------------------------------------------------------- layout
+
+def layout(topk_idx: np.ndarray, num_experts: int, num_ranks: int):
+    ti = _c(topk_idx, np.int64)
+    T, K = ti.shape
+    ntpr = np.zeros(num_ranks, np.int32)
+    ntpe = np.zeros(num_experts, np.int32)
+    itr = np.zeros((T, num_ranks), np.uint8)
+    st = lib().oracle_layout(_ptr(ti), T, K, num_experts, num_ranks, _ptr(ntpr), _ptr(ntpe), _ptr(itr))
+    if st:
+        raise OracleError(st, "layout")
+    return {"num_tokens_per_rank": ntpr, "num_tokens_per_expert": ntpe,
+            "is_token_in_rank": itr.astype(bool)}
+
+
+def capacity_bound(T: int, K: int, E: int, A: int) -> int:
+    return T * K + E * (A - 1)
+
+
+def slots(topk_idx, topk_weights, num_experts: int, num_ranks: int, expert_alignment: int = 1,
+          capacity: Optional[int] = None):
+    ti = _c(topk_idx, np.int64)
+    tw = _c(topk_weights, np.float32)
+    T, K = ti.shape
+    E, A = num_experts, expert_alignment
+    cap = capacity_bound(T, K, E, A) if capacity is None else capacity
+    psum = np.zeros(E, np.int32)
+    cnt = np.zeros(E, np.int32)
+    dst = np.zeros((T, K), np.int32)
+    meta = np.zeros((max(cap, 1), 2), np.int32)
+    rti = np.zeros((max(cap, 1), K), np.int32)
+    rtw = np.zeros((max(cap, 1), K), np.float32)
+    n = C.c_int64(0)
+    st = lib().oracle_slots(_ptr(ti), _ptr(tw), T, K, E, num_ranks, A, cap, _ptr(psum), _ptr(cnt),
+                            _ptr(dst), _ptr(meta), _ptr(rti), _ptr(rtw), C.byref(n))
+    if st:
+        raise OracleError(st, "slots")
+    nr = n.value
+    return {"psum_num_recv_tokens_per_expert": psum, "num_recv_tokens_per_expert": cnt,
+            "dst_buffer_slot_idx": dst, "recv_src_metadata": meta[:nr],
+            "recv_topk_idx": rti[:nr], "recv_topk_weights": rtw[:nr], "num_recv_rows": nr}
+
+
+def quantize_row(x_row: np.ndarray, quant: str, quant_size: int, round_scale: bool):
+    xr = _c(x_row, np.uint16)
+    H = xr.shape[0]
+    q = np.zeros(H, np.uint8)
+    sc = np.zeros(H // quant_size, np.float32)
+    st = lib().oracle_quantize_row(_ptr(xr), H, QUANT[quant], quant_size, int(round_scale), _ptr(q), _ptr(sc))
+    if st:
+        raise OracleError(st, "quantize_row")
+    return q, sc
+
+
+def dispatch_rows(x, dst_buffer_slot_idx, quant: str = "none", quant_size: int = 128,
+                  round_scale: bool = False, tokens=None, num_rows: Optional[int] = None,
+                  out=None):
+    """recv_x (and recv_scales) rows of the listed tokens.
+
+    Rows of tokens not listed keep their previous content (zero when the
+    buffers are allocated here, or the caller's ``out`` = (recv_x, recv_scales)).
+    """
+    xs = _c(x, np.uint16)
+    dst = _c(dst_buffer_slot_idx, np.int32)
+    T, H = xs.shape
+    K = dst.shape[1]
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tok = _c(tokens, np.int32)
+    if out is None:
+        rows = int(dst.max()) + 1 if num_rows is None else num_rows
+        rows = max(rows, 0)
+        if quant == "none":
+            recv_x = np.zeros((rows, H), np.uint16)
+            recv_scales = None
+        else:
+            recv_x = np.zeros((rows, H), np.uint8)
+            recv_scales = np.zeros((rows, H // quant_size), np.float32)
+    else:
+        recv_x, recv_scales = out
+        rows = recv_x.shape[0]
+    st = lib().oracle_dispatch_rows(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size,
+                                    int(round_scale), _ptr(tok), tok.shape[0], _ptr(recv_x),
+                                    _ptr(recv_scales), rows)
+    if st:
+        raise OracleError(st, "dispatch_rows")
+    return recv_x, recv_scales
+
+
+def combine_rows(y, dst_buffer_slot_idx, topk_weights, tokens=None):
+    ys = _c(y, np.uint16)
+    dst = _c(dst_buffer_slot_idx, np.int32)
+    tw = _c(topk_weights, np.float32)
+    T, K = dst.shape
+    H = ys.shape[1]
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tok = _c(tokens, np.int32)
+    out = np.zeros((tok.shape[0], H), np.uint16)
+    st = lib().oracle_combine_rows(_ptr(ys), ys.shape[0], H, T, K, _ptr(dst), _ptr(tw), _ptr(tok),
+                                   tok.shape[0], _ptr(out))
+    if st:
+        raise OracleError(st, "combine_rows")
+    return out
+
+
+def round_tokens(T: int, R: int, rounds: int, j: int) -> np.ndarray:
+    out = np.zeros(max(T // max(rounds, 1), 1), np.int32)
+    n = lib().oracle_round_tokens(T, R, rounds, j, _ptr(out))
+    if n < 0:
+        raise OracleError(INVALID_ARG, "round_tokens")
+    return out[:n]
+
+
+def dispatch(x, topk_idx, topk_weights, num_experts: int, num_ranks: int,
+             expert_alignment: int = 1, quant: str = "none", quant_size: int = 128,
+             round_scale: bool = False, num_rounds: int = 1):
+    """Full dispatch: slots over all tokens, then the rows, round by round."""
+    s = slots(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment)
+    T = np.asarray(topk_idx).shape[0]
+    recv_x, recv_scales = dispatch_rows(x, s["dst_buffer_slot_idx"], quant, quant_size,
+                                        round_scale, tokens=np.zeros(0, np.int32),
+                                        num_rows=s["num_recv_rows"])
+    for j in range(num_rounds):
+        tok = round_tokens(T, num_ranks, num_rounds, j) if num_rounds > 1 else None
+        dispatch_rows(x, s["dst_buffer_slot_idx"], quant, quant_size, round_scale,
+                      tokens=tok, out=(recv_x, recv_scales))
+    s["recv_x"] = recv_x
+    s["recv_scales"] = recv_scales
+    return s
+
+
+def combine(y, dst_buffer_slot_idx, topk_weights, num_ranks: int = 1, num_rounds: int = 1):
+    T = np.asarray(dst_buffer_slot_idx).shape[0]
+    if num_rounds == 1:
+        return combine_rows(y, dst_buffer_slot_idx, topk_weights)
+    H = np.asarray(y).shape[1]
+    out = np.zeros((T, H), np.uint16)
+    for j in range(num_rounds):
+        tok = round_tokens(T, num_ranks, num_rounds, j)
+        out[tok] = combine_rows(y, dst_buffer_slot_idx, topk_weights, tokens=tok)
+    return out

@@ -1,0 +1,372 @@
+/*
+ * ep_oracle.c -- CPU oracle for MoE expert-parallel dispatch / combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is a plain, slow, single-threaded reference
+ * that the parity tests, the smoke check and the benchmark's CPU-baseline leg
+ * compare the CUDA path against.  It shares no code, header, table or helper
+ * with the CUDA library, and the product path never calls it.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - get_dispatch_layout: num_tokens_per_rank, num_tokens_per_expert and
+ *    is_token_in_rank from topk_idx ("DeepEP V1 vs V2 comparative analysis",
+ *    section 2.1, the V1 normal-mode API).  Expert e lives on rank e / L with
+ *    L = num_local_experts = num_experts / ep_world_size ("DeepEP on Ascend A2"
+ *    page, Usage, the HCCL_BUFFSIZE note).  Entries equal to -1 are masked.
+ *  - dispatch slots: one received row per unmasked (token, expert) pair
+ *    (expand mode, do_expand in the EPHandle fields of section 3.1 of the
+ *    comparative analysis), rows ordered by (expert, source token, k) -- the
+ *    deterministic order of section 8.4 -- and every expert segment rounded up
+ *    to expert_alignment (section 3.1).  psum_num_recv_tokens_per_expert is the
+ *    inclusive prefix sum of the aligned counts; the unaligned counts are
+ *    returned beside it (section 3.1; the A2 page's MOE_EXPERT_TOKEN_NUMS_TYPE
+ *    switch between counts and prefix sums).  recv_src_metadata and
+ *    dst_buffer_slot_idx are the two directions of the row <-> (token, k) map.
+ *  - recv_x: the bf16 row of the source token, or its quantisation:
+ *    FP8 e4m3 with one fp32 scale per 128 channels, optionally rounded up to a
+ *    power of two (use_fp8 / round_scale / use_ue8m0 of low_latency_dispatch in
+ *    "DeepEP communication library guide v2.1"; float8_e4m3fn storage in
+ *    section 7.4 of the comparative analysis), or int8 with quant_size 128
+ *    (group) or hidden (per token) (guide v2.1, section 1.3.1; the A2 page's
+ *    DEEP_NORMAL_MODE_USE_INT8_QUANT).
+ *  - combine: out[t] = bf16( sum over unmasked k, in k order, of
+ *    topk_weights[t,k] * y[dst_buffer_slot_idx[t,k]] ), accumulated in fp32
+ *    with fused multiply-add (the reverse of dispatch, combine in section 9.2
+ *    of the comparative analysis).
+ *  - long-sequence rounds: the A2 page's "ant moving home" feature processes
+ *    each rank's tokens in rounds of PER_ROUND_TOKENS; the API is unchanged, so
+ *    the result equals the one-shot result (see oracle_dispatch_rows with a
+ *    round token list).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ * padding rows hold zero bytes, scale 0, metadata (-1, -1), recv_topk_idx -1
+ * and weight 0; the FP8/int8 amax is floored at 1e-4; scale = amax / 448 (or
+ * / 127) by IEEE fp32 division; x / scale by IEEE fp32 division; FP8 encoding
+ * rounds to nearest even and saturates to +-448; int8 rounds to nearest even
+ * and clamps to [-127, 127]; recv_topk_idx holds the receiving rank's local
+ * expert id of every top-k entry that lives on that rank, else -1.
+ *
+ * Status codes are this file's own (0 ok, 1 invalid argument, 2 expert id out
+ * of range, 3 receive capacity too small).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_INVALID_ARG 1
+#define OR_BAD_EXPERT_ID 2
+#define OR_CAPACITY 3
+
+#define OR_QUANT_NONE 0
+#define OR_QUANT_FP8 1
+#define OR_QUANT_INT8 2
+
+/* ---------------------------------------------------------------- numbers */
+
+/* bf16 is the upper half of an IEEE-754 binary32. */
+float oracle_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a binary32 to the nearest bf16, ties to even (NaN stays NaN). */
+uint16_t oracle_f32_to_bf16(float f) {
+    if (isnan(f)) return 0x7fc0;
+    double v = (double)f;                  /* exact */
+    if (v == 0.0 || isinf(v)) {
+        uint32_t u;
+        memcpy(&u, &f, sizeof u);
+        return (uint16_t)(u >> 16);
+    }
+    /* bf16 keeps 8 significant bits: quantum of the binade of |v| is
+     * 2^(floor(log2|v|) - 7), or 2^-133 below the smallest normal 2^-126. */
+    int ex;
+    frexp(fabs(v), &ex);                   /* |v| = m * 2^ex, m in [0.5, 1) */
+    int e2 = ex - 1;
+    if (e2 < -126) e2 = -126;
+    double q = ldexp(1.0, e2 - 7);
+    double n = nearbyint(fabs(v) / q);     /* exact quotient; ties to even */
+    double r = n * q;
+    float rf = (float)r;                   /* exact unless it overflows to inf */
+    uint32_t u;
+    memcpy(&u, &rf, sizeof u);
+    uint16_t bits = (uint16_t)(u >> 16);
+    return v < 0 ? (uint16_t)(bits | 0x8000) : bits;
+}
+
+/* OCP 8-bit floating point, E4M3 ("fn": finite values and NaN only):
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+ * is subnormal (m * 2^-9); S.1111.111 is NaN; the largest finite value is
+ * 1.75 * 2^8 = 448. */
+double oracle_e4m3_to_f64(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    return s ? -v : v;
+}
+
+/* binary32 -> E4M3, round to nearest even, saturating to +-448 (NaN -> NaN). */
+uint8_t oracle_f32_to_e4m3(float x) {
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    uint8_t sign = (uint8_t)((u >> 24) & 0x80);
+    if (isnan(x)) return (uint8_t)(sign | 0x7f);
+    double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7e);
+    if (a == 0.0) return sign;
+    int ex;
+    frexp(a, &ex);
+    int e2 = ex - 1;                                   /* 2^e2 <= a < 2^(e2+1) */
+    double q = (e2 < -6) ? ldexp(1.0, -9) : ldexp(1.0, e2 - 3); /* spacing */
+    double v = nearbyint(a / q) * q;                   /* nearest, ties even */
+    if (v == 0.0) return sign;
+    if (v < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)(v / ldexp(1.0, -9)));
+    frexp(v, &ex);
+    e2 = ex - 1;
+    int m = (int)(v / ldexp(1.0, e2 - 3)) - 8;         /* 0..7 */
+    return (uint8_t)(sign | ((e2 + 7) << 3) | m);
+}
+
+/* 2^ceil(log2 s) for a positive normal s (the ue8m0 power-of-two scale). */
+float oracle_pow2_ceil(float s) {
+    int ex;
+    double m = frexp((double)s, &ex);                  /* s = m * 2^ex */
+    if (m == 0.5) return s;                            /* already 2^(ex-1) */
+    return (float)ldexp(1.0, ex);
+}
+
+/* ---------------------------------------------------------------- layout */
+
+static int check_ids(const int64_t* topk_idx, int T, int K, int E) {
+    for (int64_t i = 0; i < (int64_t)T * K; ++i)
+        if (topk_idx[i] < -1 || topk_idx[i] >= E) return OR_BAD_EXPERT_ID;
+    return OR_OK;
+}
+
+/* get_dispatch_layout on one GPU (the RDMA-rank output has no meaning here).
+ * num_tokens_per_expert[e] = #{(t,k) : topk_idx[t,k] == e};
+ * is_token_in_rank[t,r]   = some unmasked k of token t has expert on rank r;
+ * num_tokens_per_rank[r]  = #{t : is_token_in_rank[t,r]}. */
+int oracle_layout(const int64_t* topk_idx, int T, int K, int E, int R,
+                  int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                  uint8_t* is_token_in_rank) {
+    if (T < 0 || K < 1 || E < 1 || R < 1 || E % R != 0) return OR_INVALID_ARG;
+    int st = check_ids(topk_idx, T, K, E);
+    if (st) return st;
+    int L = E / R;
+    memset(num_tokens_per_rank, 0, sizeof(int32_t) * R);
+    memset(num_tokens_per_expert, 0, sizeof(int32_t) * E);
+    memset(is_token_in_rank, 0, (size_t)T * R);
+    for (int t = 0; t < T; ++t)
+        for (int k = 0; k < K; ++k) {
+            int64_t e = topk_idx[(int64_t)t * K + k];
+            if (e < 0) continue;
+            num_tokens_per_expert[e] += 1;
+            is_token_in_rank[(int64_t)t * R + e / L] = 1;
+        }
+    for (int t = 0; t < T; ++t)
+        for (int r = 0; r < R; ++r) num_tokens_per_rank[r] += is_token_in_rank[(int64_t)t * R + r];
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------ slot order */
+
+/* Assigns every unmasked (t,k) its received row.  Experts are visited in
+ * order e = 0..E-1 (so ranks too, experts being rank-contiguous); within an
+ * expert, tokens in ascending t (= source rank, then its local index), then
+ * ascending k.  Each expert's segment is padded to a multiple of A.
+ * Rows [0, n_al) of the per-row outputs are written; capacity rows are
+ * needed (else OR_CAPACITY and nothing is written). */
+int oracle_slots(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R,
+                 int A, int64_t capacity,
+                 int32_t* psum_num_recv_tokens_per_expert,   /* [E] inclusive, aligned */
+                 int32_t* num_recv_tokens_per_expert,        /* [E] unaligned */
+                 int32_t* dst_buffer_slot_idx,               /* [T,K] */
+                 int32_t* recv_src_metadata,                 /* [cap,2] (t,k) */
+                 int32_t* recv_topk_idx,                     /* [cap,K] */
+                 float* recv_topk_weights,                   /* [cap,K] */
+                 int64_t* num_recv_rows) {
+    if (T < 0 || K < 1 || E < 1 || R < 1 || E % R != 0 || A < 1) return OR_INVALID_ARG;
+    int st = check_ids(topk_idx, T, K, E);
+    if (st) return st;
+    int L = E / R;
+    int64_t* count = calloc((size_t)E, sizeof(int64_t));
+    for (int64_t i = 0; i < (int64_t)T * K; ++i)
+        if (topk_idx[i] >= 0) count[topk_idx[i]] += 1;
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) {
+        int64_t aligned = (count[e] + A - 1) / A * A;
+        total += aligned;
+        psum_num_recv_tokens_per_expert[e] = (int32_t)total;
+        num_recv_tokens_per_expert[e] = (int32_t)count[e];
+    }
+    *num_recv_rows = total;
+    free(count);
+    if (total > capacity) return OR_CAPACITY;
+
+    for (int64_t i = 0; i < (int64_t)T * K; ++i) dst_buffer_slot_idx[i] = -1;
+    for (int64_t row = 0; row < total; ++row) {
+        recv_src_metadata[2 * row] = -1;
+        recv_src_metadata[2 * row + 1] = -1;
+        for (int j = 0; j < K; ++j) {
+            recv_topk_idx[row * K + j] = -1;
+            recv_topk_weights[row * K + j] = 0.0f;
+        }
+    }
+    int64_t seg_start = 0;
+    for (int e = 0; e < E; ++e) {
+        int64_t row = seg_start;
+        int r_dst = e / L;
+        for (int t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k) {
+                if (topk_idx[(int64_t)t * K + k] != e) continue;
+                dst_buffer_slot_idx[(int64_t)t * K + k] = (int32_t)row;
+                recv_src_metadata[2 * row] = t;
+                recv_src_metadata[2 * row + 1] = k;
+                for (int j = 0; j < K; ++j) {
+                    int64_t ej = topk_idx[(int64_t)t * K + j];
+                    if (ej >= 0 && ej / L == r_dst) {
+                        recv_topk_idx[row * K + j] = (int32_t)(ej - (int64_t)r_dst * L);
+                        recv_topk_weights[row * K + j] = topk_weights[(int64_t)t * K + j];
+                    }
+                }
+                row += 1;
+            }
+        seg_start = psum_num_recv_tokens_per_expert[e];   /* padding rows stay (-1,...) */
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------- quantisation */
+
+/* Quantises one bf16 row of H channels.  quant: OR_QUANT_FP8 or OR_QUANT_INT8;
+ * quant_size: channels per scale (128, or H for one scale per token).
+ * q receives H bytes (e4m3 codes or int8), scales H / quant_size floats. */
+int oracle_quantize_row(const uint16_t* x, int H, int quant, int quant_size, int round_scale,
+                        uint8_t* q, float* scales) {
+    if (quant != OR_QUANT_FP8 && quant != OR_QUANT_INT8) return OR_INVALID_ARG;
+    if (quant_size < 1 || H % quant_size != 0) return OR_INVALID_ARG;
+    const float qmax = (quant == OR_QUANT_FP8) ? 448.0f : 127.0f;
+    for (int g = 0; g < H / quant_size; ++g) {
+        float amax = 0.0f;
+        for (int i = 0; i < quant_size; ++i) {
+            float v = fabsf(oracle_bf16_to_f32(x[g * quant_size + i]));
+            if (v > amax) amax = v;
+        }
+        if (amax < 1e-4f) amax = 1e-4f;
+        float s = amax / qmax;
+        if (round_scale) s = oracle_pow2_ceil(s);
+        scales[g] = s;
+        for (int i = 0; i < quant_size; ++i) {
+            float v = oracle_bf16_to_f32(x[g * quant_size + i]) / s;
+            if (quant == OR_QUANT_FP8) {
+                q[g * quant_size + i] = oracle_f32_to_e4m3(v);
+            } else {
+                float r = nearbyintf(v);
+                if (r > 127.0f) r = 127.0f;
+                if (r < -127.0f) r = -127.0f;
+                q[g * quant_size + i] = (uint8_t)(int8_t)r;
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------- dispatch */
+
+/* Writes the received rows of the listed tokens: recv_x[dst_buffer_slot_idx[t,k]]
+ * = x[t] (bf16 bits) or its quantisation, computed once per source token and
+ * copied to each of its rows.  recv_x rows are H*esize bytes (esize 2 for bf16,
+ * 1 for fp8/int8); recv_scales rows are H/quant_size floats (quantised only). */
+int oracle_dispatch_rows(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
+                         int quant, int quant_size, int round_scale,
+                         const int32_t* tokens, int64_t n_tokens,
+                         uint8_t* recv_x, float* recv_scales, int64_t capacity) {
+    if (H < 1) return OR_INVALID_ARG;
+    int esize = (quant == OR_QUANT_NONE) ? 2 : 1;
+    int ns = (quant == OR_QUANT_NONE) ? 0 : H / quant_size;
+    uint8_t* q = malloc((size_t)H);
+    float* sc = malloc(sizeof(float) * (size_t)(ns > 0 ? ns : 1));
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int t = tokens[i];
+        if (t < 0 || t >= T) { free(q); free(sc); return OR_INVALID_ARG; }
+        const uint16_t* xr = x + (int64_t)t * H;
+        if (quant != OR_QUANT_NONE) {
+            int st = oracle_quantize_row(xr, H, quant, quant_size, round_scale, q, sc);
+            if (st) { free(q); free(sc); return st; }
+        }
+        for (int k = 0; k < K; ++k) {
+            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+            if (row < 0) continue;
+            if (row >= capacity) { free(q); free(sc); return OR_CAPACITY; }
+            uint8_t* dst = recv_x + row * H * esize;
+            if (quant == OR_QUANT_NONE) {
+                memcpy(dst, xr, (size_t)H * 2);
+            } else {
+                memcpy(dst, q, (size_t)H);
+                memcpy(recv_scales + row * ns, sc, sizeof(float) * ns);
+            }
+        }
+    }
+    free(q);
+    free(sc);
+    return OR_OK;
+}
+
+/* -------------------------------------------------------------- combine */
+
+/* out[i] = bf16( fma chain over k = 0..K-1 with dst_buffer_slot_idx[t,k] >= 0 of
+ * topk_weights[t,k] * y[slot] ), starting from +0.0f, for t = tokens[i].
+ * out is [n_tokens, H] (compact, in list order). */
+int oracle_combine_rows(const uint16_t* y, int64_t y_rows, int H, int T, int K,
+                        const int32_t* dst_buffer_slot_idx, const float* topk_weights,
+                        const int32_t* tokens, int64_t n_tokens, uint16_t* out) {
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int t = tokens[i];
+        if (t < 0 || t >= T) return OR_INVALID_ARG;
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+                if (row < 0) continue;
+                if (row >= y_rows) return OR_CAPACITY;
+                acc = fmaf(topk_weights[(int64_t)t * K + k], oracle_bf16_to_f32(y[row * H + h]), acc);
+            }
+            out[i * H + h] = oracle_f32_to_bf16(acc);
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------- long sequences */
+
+/* Token list of round j of the "ant moving home" schedule: each of the R
+ * source ranks owns T/R consecutive tokens and sends its j-th block of
+ * (T/R)/rounds tokens in round j.  Returns the number of tokens written. */
+int64_t oracle_round_tokens(int T, int R, int rounds, int j, int32_t* tokens) {
+    if (R < 1 || rounds < 1 || T % R != 0 || (T / R) % rounds != 0 || j < 0 || j >= rounds)
+        return -1;
+    int tpr = T / R, per_round = tpr / rounds;
+    int64_t n = 0;
+    for (int r = 0; r < R; ++r)
+        for (int i = 0; i < per_round; ++i) tokens[n++] = r * tpr + j * per_round + i;
+    return n;
+}
+
+/* ------------------------------------------------- array forms (for tests) */
+
+void oracle_f32_to_e4m3_n(const float* x, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_e4m3(x[i]);
+}
+
+void oracle_f32_to_bf16_n(const float* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(x[i]);
+}
+
+void oracle_e4m3_to_f64_n(const uint8_t* c, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_to_f64(c[i]);
+}
