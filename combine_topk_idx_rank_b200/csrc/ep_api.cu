@@ -1,0 +1,265 @@
+// C ABI of libep.so (declared in include/ep.h): argument validation,
+// workspace carving and the launch sequence of each call.  Stateless: every
+// buffer belongs to the caller, nothing is allocated here.
+#include <stdio.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool sizes_ok(int32_t T, int32_t K, int32_t E, int32_t R) {
+    if (T < 0 || T > (1 << 24)) return false;
+    if (K < 1 || K > kMaxTopk) return false;
+    if (E < 1 || E > kMaxExperts) return false;
+    if (R < 1 || R > kMaxRanks || E % R != 0) return false;
+    if (T % R != 0) return false;
+    return true;
+}
+
+ep_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return EP_OK;
+    fprintf(stderr, "libep: CUDA error %d (%s)\n", (int)e, cudaGetErrorString(e));
+    return EP_ERR_CUDA;
+}
+
+struct WsPtrs {
+    int32_t* hdr;
+    int32_t* counts;
+    int32_t* rank_counts;
+    int32_t* pad_base;
+    int32_t* pad_start;
+    int32_t* chunk_off;
+};
+
+WsPtrs carve(void* ws, const WsLayout& L) {
+    char* b = static_cast<char*>(ws);
+    return WsPtrs{reinterpret_cast<int32_t*>(b + L.hdr), reinterpret_cast<int32_t*>(b + L.counts),
+                  reinterpret_cast<int32_t*>(b + L.rank_counts), reinterpret_cast<int32_t*>(b + L.pad_base),
+                  reinterpret_cast<int32_t*>(b + L.pad_start), reinterpret_cast<int32_t*>(b + L.chunk_off)};
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" {
+
+int64_t ep_recv_capacity_bound(int32_t T, int32_t K, int32_t E, int32_t A) {
+    if (T < 0 || K < 1 || E < 1 || A < 1) return 0;
+    return (int64_t)T * K + (int64_t)E * (A - 1);
+}
+
+size_t ep_workspace_bytes(int32_t T, int32_t K, int32_t E, int32_t R) {
+    if (!sizes_ok(T, K, E, R)) return 0;
+    return ws_layout(T, K, E, R).total;
+}
+
+const char* ep_status_string(ep_status_t s) {
+    switch (s) {
+        case EP_OK: return "ok";
+        case EP_ERR_INVALID_ARG: return "invalid argument";
+        case EP_ERR_BAD_EXPERT_ID: return "expert id out of range";
+        case EP_ERR_CAPACITY: return "receive capacity too small";
+        case EP_ERR_CUDA: return "CUDA error";
+        case EP_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E,
+                                   int32_t R, int32_t* num_tokens_per_rank,
+                                   int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                                   int32_t* err, void* ws, size_t ws_bytes, void* stream) {
+    if (!sizes_ok(T, K, E, R) || err == nullptr || ws == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && topk_idx == nullptr) return EP_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, K, E, R);
+    if (ws_bytes < L.total) return EP_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsPtrs w = carve(ws, L);
+    ep_status_t s = cuda_status(cudaMemsetAsync(ws, 0, L.zero_bytes, st));
+    if (s) return s;
+    if (T > 0) {
+        LayoutArgs la{topk_idx, T, K, E, R, E / R, nullptr, nullptr, is_token_in_rank, nullptr,
+                      w.counts, w.rank_counts, w.hdr};
+        s = cuda_status(launch_layout(la, L.nchunks, st));
+        if (s) return s;
+    }
+    ScanArgs sa{};
+    sa.E = E; sa.R = R; sa.A = 1; sa.nchunks = L.nchunks;
+    sa.capacity = 0; sa.check_capacity = 0;
+    sa.counts = w.counts; sa.rank_counts = w.rank_counts; sa.layout_err = w.hdr;
+    sa.chunk_off = nullptr; sa.pad_base = nullptr; sa.pad_start = nullptr; sa.hdr = w.hdr;
+    sa.num_tokens_per_expert = num_tokens_per_expert;
+    sa.num_tokens_per_rank = num_tokens_per_rank;
+    sa.err_out = err;
+    return cuda_status(launch_scan(sa, st));
+}
+
+ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                        const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                        const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                        int32_t* recv_topk_idx, float* recv_topk_weights,
+                        int64_t recv_capacity, ep_handle_t* h,
+                        int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                        uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream) {
+    if (!sizes_ok(T, K, E, R) || opts == nullptr || h == nullptr) return EP_ERR_INVALID_ARG;
+    if (H < 8 || H > 65536 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    const int A = opts->expert_alignment;
+    const int quant = opts->quant;
+    const int rounds = opts->num_rounds;
+    if (A < 1 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
+    if (ep_recv_capacity_bound(T, K, E, A) >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
+    if (recv_capacity < 0 || recv_capacity >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8)
+        return EP_ERR_INVALID_ARG;
+    int quant_size = 0;
+    if (quant != EP_QUANT_NONE) {
+        quant_size = opts->quant_size;
+        const bool group = quant_size == 16 || quant_size == 32 || quant_size == 64 ||
+                           quant_size == 128 || quant_size == 256 || quant_size == 512;
+        if (H % 16 != 0 || !(quant_size == H || group) || H % quant_size != 0) return EP_ERR_INVALID_ARG;
+        if (recv_scales == nullptr) return EP_ERR_INVALID_ARG;
+    }
+    if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
+        h->recv_src_metadata == nullptr || h->dst_buffer_slot_idx == nullptr || h->err == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (recv_capacity > 0 && (recv_x == nullptr || recv_topk_idx == nullptr || recv_topk_weights == nullptr))
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || topk_idx == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, K, E, R);
+    if (ws == nullptr || ws_bytes < L.total) return EP_ERR_INVALID_ARG;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsPtrs w = carve(ws, L);
+    h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
+    h->hidden = H; h->expert_alignment = A; h->num_rounds = rounds; h->recv_capacity = recv_capacity;
+
+    ep_status_t s = cuda_status(cudaMemsetAsync(ws, 0, L.zero_bytes, st));
+    if (s) return s;
+    if (T > 0) {
+        LayoutArgs la{topk_idx, T, K, E, R, E / R, h->dst_buffer_slot_idx, w.chunk_off,
+                      is_token_in_rank, h->topk_idx, w.counts, w.rank_counts, w.hdr};
+        s = cuda_status(launch_layout(la, L.nchunks, st));
+        if (s) return s;
+    }
+    ScanArgs sa{};
+    sa.E = E; sa.R = R; sa.A = A; sa.nchunks = L.nchunks;
+    sa.capacity = recv_capacity; sa.check_capacity = 1;
+    sa.counts = w.counts; sa.rank_counts = w.rank_counts; sa.layout_err = w.hdr;
+    sa.chunk_off = T > 0 ? w.chunk_off : nullptr;
+    sa.pad_base = w.pad_base; sa.pad_start = w.pad_start; sa.hdr = w.hdr;
+    sa.psum = h->psum_num_recv_tokens_per_expert;
+    sa.num_recv = h->num_recv_tokens_per_expert;
+    sa.num_tokens_per_expert = num_tokens_per_expert;
+    sa.num_tokens_per_rank = num_tokens_per_rank;
+    sa.cumulative = opts->cumulative_local_expert_recv_stats;
+    sa.err_out = h->err;
+    s = cuda_status(launch_scan(sa, st));
+    if (s) return s;
+
+    if (opts->event_pack_begin) {
+        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
+        if (s) return s;
+    }
+    if (T > 0) {
+        const int tpr = T / R, per_round = tpr / rounds;
+        for (int j = 0; j < rounds; ++j) {
+            PackArgs pa{};
+            pa.x = static_cast<const uint16_t*>(x);
+            pa.T = T; pa.H = H; pa.K = K; pa.E = E; pa.L = E / R;
+            pa.topk_idx = topk_idx; pa.topk_weights = topk_weights;
+            pa.dst_slot = h->dst_buffer_slot_idx; pa.chunk_off = w.chunk_off;
+            pa.recv_x = static_cast<uint8_t*>(recv_x); pa.recv_scales = recv_scales;
+            pa.recv_topk_idx = recv_topk_idx; pa.recv_topk_weights = recv_topk_weights;
+            pa.recv_meta = h->recv_src_metadata; pa.capacity = recv_capacity;
+            pa.pad_base = w.pad_base; pa.pad_start = w.pad_start; pa.hdr = w.hdr;
+            pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
+            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
+            pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
+            s = cuda_status(launch_pack(pa, quant, st));
+            if (s) return s;
+        }
+    }
+    if (opts->event_pack_end) {
+        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_end), st));
+        if (s) return s;
+    }
+    return EP_OK;
+}
+
+ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_weights, void* out,
+                       void* stream) {
+    if (h == nullptr) return EP_ERR_INVALID_ARG;
+    const int T = h->num_tokens, K = h->num_topk, H = h->hidden, R = h->num_ranks;
+    const int rounds = h->num_rounds;
+    if (!sizes_ok(T, K, h->num_experts, R)) return EP_ERR_INVALID_ARG;
+    if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
+    if (h->dst_buffer_slot_idx == nullptr || h->err == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (out == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
+    if (h->recv_capacity > 0 && y == nullptr) return EP_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out)) return EP_ERR_INVALID_ARG;
+    if (T == 0) return EP_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int tpr = T / R, per_round = tpr / rounds;
+    for (int j = 0; j < rounds; ++j) {
+        CombineArgs ca{};
+        ca.y = static_cast<const uint16_t*>(y); ca.y_rows = h->recv_capacity;
+        ca.H = H; ca.K = K; ca.T = T;
+        ca.dst_slot = h->dst_buffer_slot_idx; ca.topk_weights = topk_weights;
+        ca.out = static_cast<uint16_t*>(out);
+        ca.tokens_per_rank = tpr; ca.per_round = per_round; ca.round = j; ca.n_items = R * per_round;
+        ca.err = h->err;
+        ep_status_t s = cuda_status(launch_combine(ca, st));
+        if (s) return s;
+    }
+    return EP_OK;
+}
+
+ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status) {
+    if (err == nullptr || host_status == nullptr) return EP_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ep_status_t s = cuda_status(cudaMemcpyAsync(host_status, err, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+    if (s) return s;
+    return cuda_status(cudaStreamSynchronize(st));
+}
+
+ep_status_t ep_copy_recv_counts(const ep_handle_t* h, void* stream, int32_t* host_counts,
+                                int64_t* num_recv_rows) {
+    if (h == nullptr || h->num_experts < 1) return EP_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t last = 0;
+    ep_status_t s;
+    if (host_counts) {
+        s = cuda_status(cudaMemcpyAsync(host_counts, h->num_recv_tokens_per_expert,
+                                        sizeof(int32_t) * h->num_experts, cudaMemcpyDeviceToHost, st));
+        if (s) return s;
+    }
+    if (num_recv_rows) {
+        s = cuda_status(cudaMemcpyAsync(&last, h->psum_num_recv_tokens_per_expert + h->num_experts - 1,
+                                        sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+        if (s) return s;
+    }
+    s = cuda_status(cudaStreamSynchronize(st));
+    if (s) return s;
+    if (num_recv_rows) *num_recv_rows = last;
+    return EP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,240 @@
+// Routing histogram (get_dispatch_layout) and the prefix scan that assigns
+// every (token, k) entry its received row in the deterministic
+// (expert, token, k) order ("DeepEP V1 vs V2 comparative analysis",
+// sections 2.1, 3.1 and 8.4), with expert segments padded to
+// expert_alignment.
+//
+// The order needs no sort: k_layout gives each entry its rank among the
+// entries of its 128-token chunk that go to the same expert (in (t,k)
+// order), and k_scan turns the per-chunk histograms into the row offset of
+// every (chunk, expert) pair.  Row = offset[chunk][e] + rank.  No CTA ever
+// waits on another.
+#include "ep_internal.cuh"
+
+namespace ep {
+
+// One CTA per chunk of kChunkTokens tokens.  Warp w owns a contiguous range
+// of the chunk's C*K entries and walks it 32 entries at a time; lanes that
+// hold the same expert find each other with __match_any_sync, so the rank of
+// an entry within its warp's range is the warp's running count for that
+// expert plus the number of lower lanes holding the same expert.  A scan over
+// the 8 per-warp histograms then makes the ranks chunk-wide.
+__global__ void __launch_bounds__(kLayoutThreads) k_layout(LayoutArgs a) {
+    extern __shared__ int32_t smem[];
+    const int E = a.E, K = a.K, R = a.R;
+    int32_t* wh = smem;                               // [8][E] per-warp running counts
+    int32_t* s_idx = wh + kLayoutWarps * E;           // [C*K] validated expert ids
+    int32_t* s_rcnt = s_idx + kChunkTokens * K;       // [R]
+    uint8_t* s_inr = reinterpret_cast<uint8_t*>(s_rcnt + R);  // [C][R]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * kChunkTokens;
+    const int nt = min(kChunkTokens, a.T - t0);
+    const int ne = nt * K;
+    const int64_t e0 = (int64_t)t0 * K;
+
+    for (int i = tid; i < kLayoutWarps * E; i += kLayoutThreads) wh[i] = 0;
+    for (int i = tid; i < R; i += kLayoutThreads) s_rcnt[i] = 0;
+    for (int i = tid; i < nt * R; i += kLayoutThreads) s_inr[i] = 0;
+    __syncthreads();
+
+    // entries per warp, a multiple of 32
+    const int per_warp = ((kChunkTokens * K / kLayoutWarps) + 31) & ~31;
+    const int nb = per_warp / 32;
+    int my_e[kMaxBatches], my_r[kMaxBatches];
+    const unsigned lt = lanemask_lt();
+#pragma unroll
+    for (int b = 0; b < kMaxBatches; ++b) {
+        my_e[b] = -1;
+        my_r[b] = 0;
+        if (b < nb) {
+            const int i = warp * per_warp + b * 32 + lane;
+            int e = -1;
+            if (i < ne) {
+                const int64_t v = a.topk_idx[e0 + i];
+                if (v < -1 || v >= E) {
+                    set_error(a.err, EP_ERR_BAD_EXPERT_ID);
+                } else {
+                    e = (int)v;
+                }
+                s_idx[i] = e;
+            }
+            const unsigned m = __match_any_sync(0xffffffffu, e);
+            int r = 0;
+            if (e >= 0) r = wh[warp * E + e] + __popc(m & lt);
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(m) - 1) wh[warp * E + e] += __popc(m);
+            __syncwarp();
+            my_e[b] = e;
+            my_r[b] = r;
+        }
+    }
+    __syncthreads();
+
+    // per-expert scan over the warps -> chunk-wide base of each warp's range
+    for (int e = tid; e < E; e += kLayoutThreads) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kLayoutWarps; ++w) {
+            const int v = wh[w * E + e];
+            wh[w * E + e] = run;
+            run += v;
+        }
+        if (a.chunk_hist) a.chunk_hist[(size_t)blockIdx.x * E + e] = run;
+        if (run) atomicAdd(&a.counts[e], run);
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int b = 0; b < kMaxBatches; ++b) {
+        if (b < nb) {
+            const int i = warp * per_warp + b * 32 + lane;
+            if (i < ne) {
+                const int e = my_e[b];
+                if (a.rank_in_chunk) a.rank_in_chunk[e0 + i] = e >= 0 ? wh[warp * E + e] + my_r[b] : -1;
+                if (a.topk_copy) a.topk_copy[e0 + i] = e;
+            }
+        }
+    }
+
+    // which ranks each token reaches
+    for (int tl = tid; tl < nt; tl += kLayoutThreads) {
+        for (int k = 0; k < K; ++k) {
+            const int e = s_idx[tl * K + k];
+            if (e >= 0) s_inr[tl * R + e / a.L] = 1;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < nt * R; i += kLayoutThreads) {
+        const uint8_t v = s_inr[i];
+        if (v) atomicAdd(&s_rcnt[i % R], 1);
+        if (a.is_token_in_rank) a.is_token_in_rank[(size_t)t0 * R + i] = v;
+    }
+    __syncthreads();
+    for (int r = tid; r < R; r += kLayoutThreads)
+        if (s_rcnt[r]) atomicAdd(&a.rank_counts[r], s_rcnt[r]);
+}
+
+// Inclusive scan of one value per thread over a block of 1024 threads.
+__device__ __forceinline__ int block_inclusive_scan_1024(int v, int* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int add = warp > 0 ? s_warp[warp - 1] : 0;
+    __syncthreads();   // s_warp may be reused by the caller
+    return v + add;
+}
+
+// Grid: ceil(E/32) CTAs of 32x32 threads.  Every CTA scans the E aligned
+// counts (one per thread) for the segment starts; CTA g then turns the
+// column of chunk histograms of experts [32g, 32g+32) into row offsets:
+// lane = expert, warp = one of 32 contiguous ranges of chunks.  CTA 0 writes
+// the per-expert outputs, the padding map and the status word.
+__global__ void __launch_bounds__(1024) k_scan(ScanArgs a) {
+    __shared__ int s_warp[32];
+    __shared__ int s_seg[kMaxExperts];
+    __shared__ int s_part[32][33];
+    __shared__ int s_total[2];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E;
+
+    const int cnt = tid < E ? a.counts[tid] : 0;
+    const int aligned = (int)(((int64_t)cnt + a.A - 1) / a.A * a.A);
+    const int incl = block_inclusive_scan_1024(aligned, s_warp);
+    const int seg = incl - aligned;
+    if (tid < E) s_seg[tid] = seg;
+    const int pad = aligned - cnt;
+    const int pad_incl = block_inclusive_scan_1024(pad, s_warp);
+
+    if (blockIdx.x == 0) {
+        if (tid == E - 1) {
+            s_total[0] = incl;
+            s_total[1] = pad_incl;
+        }
+        if (tid < E) {
+            if (a.psum) a.psum[tid] = incl;
+            if (a.num_recv) a.num_recv[tid] = cnt;
+            if (a.num_tokens_per_expert) a.num_tokens_per_expert[tid] = cnt;
+            if (a.cumulative) a.cumulative[tid] += cnt;
+            if (a.pad_base) a.pad_base[tid] = pad_incl - pad;
+            if (a.pad_start) a.pad_start[tid] = seg + cnt;
+        }
+        if (tid < a.R && a.num_tokens_per_rank) a.num_tokens_per_rank[tid] = a.rank_counts[tid];
+        __syncthreads();
+        if (tid == 0) {
+            const int rows = s_total[0], pads = s_total[1];
+            if (a.pad_base) a.pad_base[E] = pads;
+            a.hdr[1] = rows;
+            a.hdr[2] = pads;
+            int status = *a.layout_err;
+            if (status == 0 && a.check_capacity && (int64_t)rows > a.capacity) status = EP_ERR_CAPACITY;
+            *a.err_out = status;
+        }
+    }
+    if (a.chunk_off == nullptr) return;
+    __syncthreads();
+
+    const int e = blockIdx.x * 32 + lane;
+    const int per = (a.nchunks + 31) / 32;
+    const int c0 = min(warp * per, a.nchunks), c1 = min(c0 + per, a.nchunks);
+    int sum = 0;
+    if (e < E)
+        for (int c = c0; c < c1; ++c) sum += a.chunk_off[(size_t)c * E + e];
+    s_part[warp][lane] = sum;
+    __syncthreads();
+    {   // warp w scans column w of s_part across the 32 chunk ranges
+        const int v = s_part[lane][warp];
+        int s = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += n;
+        }
+        __syncthreads();
+        s_part[lane][warp] = s - v;
+    }
+    __syncthreads();
+    if (e < E) {
+        int run = s_seg[e] + s_part[warp][lane];
+        for (int c = c0; c < c1; ++c) {
+            const int h = a.chunk_off[(size_t)c * E + e];
+            a.chunk_off[(size_t)c * E + e] = run;
+            run += h;
+        }
+    }
+}
+
+cudaError_t launch_layout(const LayoutArgs& a, int nchunks, cudaStream_t st) {
+    const size_t smem = sizeof(int32_t) * (kLayoutWarps * a.E + kChunkTokens * a.K + a.R) +
+                        (size_t)kChunkTokens * a.R;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_layout, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_layout<<<nchunks, kLayoutThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st) {
+    const int grid = a.chunk_off ? (a.E + 31) / 32 : 1;
+    k_scan<<<grid, 1024, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

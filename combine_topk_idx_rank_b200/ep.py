@@ -1,0 +1,308 @@
+"""Python binding of libep.so: argument marshalling only.
+
+Every step of dispatch and combine runs in the library's sm_100a kernels;
+torch provides device memory and the current CUDA stream.  There is no CPU
+fallback: if libep.so is missing or cannot be loaded, importing this module
+raises.
+
+API (after the DeepEP calls described in "DeepEP V1 vs V2 comparative
+analysis", sections 2-3, and the quantisation flags of "DeepEP communication
+library guide v2.1"):
+
+    ep_get_dispatch_layout(topk_idx, num_experts, num_ranks)
+        -> (num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank)
+    ep_dispatch(x, topk_idx, topk_weights, expert_alignment=1, quant=None, *,
+                num_experts, num_ranks, ...)
+        -> (recv_x, recv_scales, recv_topk_idx, recv_topk_weights, handle)
+    ep_combine(y, handle, topk_weights) -> combined tokens [T, H] bf16
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+import os
+from typing import List, Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(HERE, "libep.so")
+
+EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, EP_ERR_TIMEOUT = range(6)
+_QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2}
+
+EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
+            "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string")
+
+
+class EPError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.ep_status_string(status).decode()} (status {status})")
+
+
+class _Opts(C.Structure):
+    _fields_ = [("expert_alignment", C.c_int32), ("quant", C.c_int32), ("quant_size", C.c_int32),
+                ("round_scale", C.c_int32), ("num_rounds", C.c_int32), ("reserved", C.c_int32),
+                ("cumulative_local_expert_recv_stats", C.c_void_p),
+                ("event_pack_begin", C.c_void_p), ("event_pack_end", C.c_void_p)]
+
+
+class _Handle(C.Structure):
+    _fields_ = [("num_tokens", C.c_int32), ("num_topk", C.c_int32), ("num_experts", C.c_int32),
+                ("num_ranks", C.c_int32), ("hidden", C.c_int32), ("expert_alignment", C.c_int32),
+                ("num_rounds", C.c_int32), ("reserved", C.c_int32), ("recv_capacity", C.c_int64),
+                ("topk_idx", C.c_void_p), ("psum_num_recv_tokens_per_expert", C.c_void_p),
+                ("num_recv_tokens_per_expert", C.c_void_p), ("recv_src_metadata", C.c_void_p),
+                ("dst_buffer_slot_idx", C.c_void_p), ("err", C.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libep.so not found at {_LIB_PATH}; build it with "
+                          "`python -m combine_topk_idx_rank_b200.build`")
+    L = C.CDLL(_LIB_PATH)
+    p, i32, i64, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+    L.ep_recv_capacity_bound.argtypes = [i32, i32, i32, i32]
+    L.ep_recv_capacity_bound.restype = i64
+    L.ep_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.ep_workspace_bytes.restype = sz
+    L.ep_get_dispatch_layout.argtypes = [p, i32, i32, i32, i32, p, p, p, p, p, sz, p]
+    L.ep_get_dispatch_layout.restype = C.c_int
+    L.ep_dispatch.argtypes = [p, i32, i32, p, p, i32, i32, i32, C.POINTER(_Opts), p, p, p, p, i64,
+                              C.POINTER(_Handle), p, p, p, p, sz, p]
+    L.ep_dispatch.restype = C.c_int
+    L.ep_combine.argtypes = [p, C.POINTER(_Handle), p, p, p]
+    L.ep_combine.restype = C.c_int
+    L.ep_read_error.argtypes = [p, p, C.POINTER(C.c_int32)]
+    L.ep_read_error.restype = C.c_int
+    L.ep_copy_recv_counts.argtypes = [C.POINTER(_Handle), p, p, C.POINTER(C.c_int64)]
+    L.ep_copy_recv_counts.restype = C.c_int
+    L.ep_status_string.argtypes = [C.c_int]
+    L.ep_status_string.restype = C.c_char_p
+    return L
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != EP_OK:
+        raise EPError(status, what)
+
+
+def recv_capacity_bound(T: int, K: int, E: int, A: int) -> int:
+    return int(_lib.ep_recv_capacity_bound(T, K, E, A))
+
+
+def workspace_bytes(T: int, K: int, E: int, R: int) -> int:
+    return int(_lib.ep_workspace_bytes(T, K, E, R))
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclasses.dataclass
+class EPHandle:
+    """Routing metadata of one dispatch, reused by combine (EPHandle)."""
+    num_tokens: int
+    num_topk: int
+    num_experts: int
+    num_ranks: int
+    hidden: int
+    expert_alignment: int
+    num_rounds: int
+    recv_capacity: int
+    topk_idx: torch.Tensor                          # [T, K] int32 copy
+    psum_num_recv_tokens_per_expert: torch.Tensor   # [E] int32
+    num_recv_tokens_per_expert: torch.Tensor        # [E] int32 (unaligned)
+    recv_src_metadata: torch.Tensor                 # [cap, 2] int32 (t, k)
+    dst_buffer_slot_idx: torch.Tensor               # [T, K] int32
+    err: torch.Tensor                               # [1] int32
+    num_recv_tokens_per_expert_list: Optional[List[int]] = None
+    num_recv_rows: Optional[int] = None
+
+    def _c(self) -> _Handle:
+        h = _Handle()
+        h.num_tokens, h.num_topk, h.num_experts = self.num_tokens, self.num_topk, self.num_experts
+        h.num_ranks, h.hidden, h.expert_alignment = self.num_ranks, self.hidden, self.expert_alignment
+        h.num_rounds, h.recv_capacity = self.num_rounds, self.recv_capacity
+        h.topk_idx = self.topk_idx.data_ptr()
+        h.psum_num_recv_tokens_per_expert = self.psum_num_recv_tokens_per_expert.data_ptr()
+        h.num_recv_tokens_per_expert = self.num_recv_tokens_per_expert.data_ptr()
+        h.recv_src_metadata = self.recv_src_metadata.data_ptr()
+        h.dst_buffer_slot_idx = self.dst_buffer_slot_idx.data_ptr()
+        h.err = self.err.data_ptr()
+        return h
+
+    def read_error(self) -> int:
+        st = C.c_int32(0)
+        _check(_lib.ep_read_error(_ptr(self.err), _stream(self.err.device), C.byref(st)), "ep_read_error")
+        return st.value
+
+    def check(self):
+        st = self.read_error()
+        if st != EP_OK:
+            raise EPError(st, "device")
+
+
+@dataclasses.dataclass
+class DispatchBuffers:
+    """Preallocated outputs of ep_dispatch for a fixed shape (reusable)."""
+    recv_x: torch.Tensor
+    recv_scales: Optional[torch.Tensor]
+    recv_topk_idx: torch.Tensor
+    recv_topk_weights: torch.Tensor
+    handle: EPHandle
+    workspace: torch.Tensor
+    quant: Optional[str]
+    quant_size: int
+
+
+def alloc_dispatch_buffers(num_tokens: int, hidden: int, num_topk: int, num_experts: int,
+                           num_ranks: int, expert_alignment: int = 1, quant: Optional[str] = None,
+                           quant_size: int = 128, num_rounds: int = 1,
+                           recv_capacity: Optional[int] = None,
+                           device: Optional[torch.device] = None) -> DispatchBuffers:
+    T, H, K, E, R, A = num_tokens, hidden, num_topk, num_experts, num_ranks, expert_alignment
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    cap = recv_capacity_bound(T, K, E, A) if recv_capacity is None else int(recv_capacity)
+    q = None if quant in (None, "none") else quant
+    if q is None:
+        recv_x = torch.empty((cap, H), dtype=torch.bfloat16, device=dev)
+        recv_scales = None
+    else:
+        recv_x = torch.empty((cap, H), dtype=torch.float8_e4m3fn if q == "fp8" else torch.int8, device=dev)
+        recv_scales = torch.empty((cap, H // quant_size), dtype=torch.float32, device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    handle = EPHandle(T, K, E, R, H, A, num_rounds, cap,
+                      topk_idx=torch.empty((T, K), **i32),
+                      psum_num_recv_tokens_per_expert=torch.empty((E,), **i32),
+                      num_recv_tokens_per_expert=torch.empty((E,), **i32),
+                      recv_src_metadata=torch.empty((max(cap, 1), 2), **i32),
+                      dst_buffer_slot_idx=torch.empty((T, K), **i32),
+                      err=torch.zeros((1,), **i32))
+    ws = torch.empty((max(workspace_bytes(T, K, E, R), 256),), dtype=torch.uint8, device=dev)
+    return DispatchBuffers(recv_x, recv_scales, torch.empty((max(cap, 1), K), **i32),
+                           torch.empty((max(cap, 1), K), dtype=torch.float32, device=dev), handle, ws,
+                           q, quant_size)
+
+
+def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int,
+                           workspace: Optional[torch.Tensor] = None, check: bool = True):
+    """Routing histogram: (num_tokens_per_rank [R] i32, num_tokens_per_expert [E] i32,
+    is_token_in_rank [T, R] bool)."""
+    _need_cuda(topk_idx, "topk_idx", torch.int64)
+    T, K = topk_idx.shape
+    dev = topk_idx.device
+    ntpr = torch.empty((num_ranks,), dtype=torch.int32, device=dev)
+    ntpe = torch.empty((num_experts,), dtype=torch.int32, device=dev)
+    itr = torch.empty((T, num_ranks), dtype=torch.bool, device=dev)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    nbytes = workspace_bytes(T, K, num_experts, num_ranks)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
+    st = _lib.ep_get_dispatch_layout(_ptr(topk_idx), T, K, num_experts, num_ranks, _ptr(ntpr), _ptr(ntpe),
+                                     _ptr(itr), _ptr(err), _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(st, "ep_get_dispatch_layout")
+    if check:
+        s = C.c_int32(0)
+        _check(_lib.ep_read_error(_ptr(err), _stream(dev), C.byref(s)), "ep_read_error")
+        if s.value:
+            raise EPError(s.value, "ep_get_dispatch_layout")
+    return ntpr, ntpe, itr
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                expert_alignment: int = 1, quant: Optional[str] = None, *, num_experts: int,
+                num_ranks: int, quant_size: int = 128, round_scale: bool = False,
+                num_rounds: int = 1, do_cpu_sync: bool = True,
+                recv_capacity: Optional[int] = None, buffers: Optional[DispatchBuffers] = None,
+                cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
+                layout_out: Optional[tuple] = None, events: Optional[tuple] = None):
+    """Dispatch: returns (recv_x, recv_scales, recv_topk_idx, recv_topk_weights, handle).
+
+    With ``do_cpu_sync`` the call waits for the GPU, checks the status word and
+    trims the outputs to the rows received (``handle.num_recv_rows``); without
+    it the outputs have ``recv_capacity`` rows and nothing waits.
+    """
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(topk_idx, "topk_idx", torch.int64)
+    _need_cuda(topk_weights, "topk_weights", torch.float32)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    if topk_idx.shape[0] != T or tuple(topk_weights.shape) != (T, K):
+        raise ValueError("x, topk_idx and topk_weights disagree on the token count / top-k")
+    q = None if quant in (None, "none") else quant
+    if q is not None and quant_size not in (16, 32, 64, 128, 256, 512, H):
+        raise ValueError(f"quant_size must be a group of 16..512 channels or hidden, got {quant_size}")
+    if buffers is None:
+        buffers = alloc_dispatch_buffers(T, H, K, num_experts, num_ranks, expert_alignment, q,
+                                         quant_size, num_rounds, recv_capacity, x.device)
+    b = buffers
+    h = b.handle
+    h.num_rounds = num_rounds
+    opts = _Opts(expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds, 0,
+                 None if cumulative_local_expert_recv_stats is None
+                 else cumulative_local_expert_recv_stats.data_ptr(),
+                 None if events is None else events[0].cuda_event,
+                 None if events is None else events[1].cuda_event)
+    ch = h._c()
+    lay = layout_out or (None, None, None)
+    stream = _stream(x.device)
+    st = _lib.ep_dispatch(_ptr(x), T, H, _ptr(topk_idx), _ptr(topk_weights), K, num_experts, num_ranks,
+                          C.byref(opts), _ptr(b.recv_x), _ptr(b.recv_scales), _ptr(b.recv_topk_idx),
+                          _ptr(b.recv_topk_weights), b.recv_x.shape[0], C.byref(ch), _ptr(lay[0]),
+                          _ptr(lay[1]), _ptr(lay[2]), _ptr(b.workspace), b.workspace.numel(), stream)
+    _check(st, "ep_dispatch")
+    h.num_tokens, h.num_topk, h.num_experts, h.num_ranks = ch.num_tokens, ch.num_topk, ch.num_experts, ch.num_ranks
+    h.hidden, h.expert_alignment, h.recv_capacity = ch.hidden, ch.expert_alignment, ch.recv_capacity
+    recv_x, recv_scales, rti, rtw = b.recv_x, b.recv_scales, b.recv_topk_idx, b.recv_topk_weights
+    if do_cpu_sync:
+        h.check()
+        counts = (C.c_int32 * num_experts)()
+        n = C.c_int64(0)
+        _check(_lib.ep_copy_recv_counts(C.byref(ch), stream, counts, C.byref(n)), "ep_copy_recv_counts")
+        h.num_recv_tokens_per_expert_list = list(counts)
+        h.num_recv_rows = n.value
+        recv_x, rti, rtw = recv_x[:n.value], rti[:n.value], rtw[:n.value]
+        if recv_scales is not None:
+            recv_scales = recv_scales[:n.value]
+    return recv_x, recv_scales, rti, rtw, h
+
+
+def ep_combine(y: torch.Tensor, handle: EPHandle, topk_weights: torch.Tensor,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Combine: out[t] = bf16(sum_k w[t,k] * y[dst_buffer_slot_idx[t,k]]), fp32 in k order."""
+    _need_cuda(y, "y", torch.bfloat16)
+    _need_cuda(topk_weights, "topk_weights", torch.float32)
+    h = handle
+    if y.shape[1] != h.hidden or y.shape[0] > h.recv_capacity:
+        raise ValueError("y must be [rows <= recv_capacity, hidden] in received-row order")
+    if tuple(topk_weights.shape) != (h.num_tokens, h.num_topk):
+        raise ValueError("topk_weights shape does not match the handle")
+    if out is None:
+        out = torch.empty((h.num_tokens, h.hidden), dtype=torch.bfloat16, device=y.device)
+    ch = h._c()
+    ch.recv_capacity = y.shape[0]
+    st = _lib.ep_combine(_ptr(y), C.byref(ch), _ptr(topk_weights), _ptr(out), _stream(y.device))
+    _check(st, "ep_combine")
+    return out

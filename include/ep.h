@@ -1,0 +1,193 @@
+/*
+ * ep.h -- C ABI of libep.so: MoE expert-parallel token dispatch and combine on
+ * one B200, with the EP ranks as logical partitions of the GPU's HBM.
+ *
+ * The calls follow the DeepEP API as the pages state it:
+ *   - ep_get_dispatch_layout  <- get_dispatch_layout(topk_idx, num_experts)
+ *     ("DeepEP V1 vs V2 comparative analysis", section 2.1);
+ *   - ep_dispatch             <- dispatch(x, topk_idx, topk_weights, ...) and
+ *     the EPHandle it returns (same page, sections 2.1, 2.2 and 3.1), with the
+ *     quantisation flags of low_latency_dispatch ("DeepEP communication
+ *     library guide v2.1", sections 1.3.1 and the API listing) and the
+ *     long-sequence rounds of the "DeepEP on Ascend A2" page;
+ *   - ep_combine              <- combine(...) (comparative analysis, section 9.2).
+ *
+ * Conventions (all calls):
+ *   - Every buffer is allocated and owned by the caller; the library keeps no
+ *     state between calls and allocates nothing.
+ *   - Pointers documented "device" must point to memory of the device that is
+ *     current on the calling thread; "host" pointers to host memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) except where stated.
+ *   - A host-side argument error returns EP_ERR_INVALID_ARG before anything
+ *     is launched.  Errors the kernels detect (an expert id out of range, a
+ *     receive capacity that is too small) are written to the device word
+ *     `err`; read it with ep_read_error.  When *err != 0 the outputs are
+ *     unspecified, but no kernel ever writes outside the buffers described
+ *     here and none waits on anything.
+ *   - Sizes: T tokens (all logical ranks together), K top-k entries per
+ *     token, E experts, R logical ranks, L = E / R local experts per rank,
+ *     H hidden channels, A expert alignment.  Token t belongs to source rank
+ *     t / (T / R); expert e lives on rank e / L.
+ *   - Limits: 1 <= K <= 16, 1 <= E <= 1024, 1 <= R <= 256, E % R == 0,
+ *     T % R == 0, 0 <= T <= 2^24, 8 <= H <= 65536 with H % 8 == 0, A >= 1,
+ *     and T*K + E*(A-1) < 2^31 rows.
+ */
+#ifndef EP_B200_EP_H
+#define EP_B200_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1,   /* rejected on the host; nothing launched */
+    EP_ERR_BAD_EXPERT_ID = 2, /* some topk_idx entry is < -1 or >= E (device) */
+    EP_ERR_CAPACITY = 3,      /* recv_capacity < rows needed (device) */
+    EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    EP_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up */
+} ep_status_t;
+
+typedef enum {
+    EP_QUANT_NONE = 0,     /* recv_x is the bf16 row, bit for bit */
+    EP_QUANT_FP8_E4M3 = 1, /* OCP e4m3fn codes, fp32 scale per quant_size channels */
+    EP_QUANT_INT8 = 2      /* int8 codes in [-127, 127], fp32 scale per quant_size */
+} ep_quant_t;
+
+/* Options of ep_dispatch. */
+typedef struct {
+    int32_t expert_alignment; /* A >= 1: each expert's segment of received rows is
+                                 padded to a multiple of A (EPHandle.expert_alignment,
+                                 comparative analysis section 3.1) */
+    int32_t quant;            /* ep_quant_t */
+    int32_t quant_size;       /* channels per scale: 128 (group) or H (per token)
+                                 (quant_size, guide v2.1 section 1.3.1); a multiple
+                                 of 16 that divides H; ignored for EP_QUANT_NONE */
+    int32_t round_scale;      /* nonzero: round each scale up to a power of two
+                                 (round_scale / use_ue8m0); stored as fp32 */
+    int32_t num_rounds;       /* >= 1, divides T / R: the rows are written in
+                                 rounds of (T/R)/num_rounds tokens per rank ("ant
+                                 moving home" long-sequence mode, Ascend A2 page);
+                                 the result equals num_rounds == 1 */
+    int32_t reserved;
+    /* optional device [E]: the unaligned per-expert counts of this call are
+     * added to it (cumulative_local_expert_recv_stats, guide v2.1) */
+    int32_t* cumulative_local_expert_recv_stats;
+    /* optional cudaEvent_t values (as void*) recorded on `stream` right before
+     * and right after the pack kernel(s), for timing; NULL = none */
+    void* event_pack_begin;
+    void* event_pack_end;
+} ep_dispatch_opts_t;
+
+/* The routing handle ep_dispatch fills and ep_combine reads (EPHandle of the
+ * comparative analysis, section 3.1).  A plain struct: the caller allocates
+ * every array (device memory), sets the pointers, and passes the same struct
+ * to ep_combine.  ep_dispatch sets the scalar fields. */
+typedef struct {
+    int32_t num_tokens, num_topk, num_experts, num_ranks, hidden, expert_alignment;
+    int32_t num_rounds, reserved;
+    int64_t recv_capacity;                       /* rows of recv_x / y */
+    int32_t* topk_idx;                           /* [T,K] copy of the routing as int32
+                                                    (-1 = masked); may be NULL */
+    int32_t* psum_num_recv_tokens_per_expert;    /* [E] inclusive prefix sum of the
+                                                    aligned per-expert counts */
+    int32_t* num_recv_tokens_per_expert;         /* [E] unaligned counts */
+    int32_t* recv_src_metadata;                  /* [recv_capacity, 2]: (t, k) of each
+                                                    received row; (-1,-1) on padding */
+    int32_t* dst_buffer_slot_idx;                /* [T,K]: row of (t,k), -1 if masked */
+    int32_t* err;                                /* [1]: device status word */
+} ep_handle_t;
+
+/* Rows ep_dispatch may need: T*K + E*(A-1) (every entry unmasked, every
+ * expert padded by A-1).  Host only. */
+int64_t ep_recv_capacity_bound(int32_t T, int32_t K, int32_t E, int32_t A);
+
+/* Bytes of device workspace the calls below need for these sizes (256-byte
+ * aligned; pass at least this many).  Host only. */
+size_t ep_workspace_bytes(int32_t T, int32_t K, int32_t E, int32_t R);
+
+/*
+ * Routing histogram (get_dispatch_layout, comparative analysis section 2.1;
+ * the RDMA-rank output has no meaning on one GPU and is not produced).
+ *   topk_idx               device int64 [T,K]; -1 = masked entry
+ *   num_tokens_per_rank    device int32 [R]: tokens with >= 1 expert on rank r
+ *   num_tokens_per_expert  device int32 [E]: (t,k) entries routed to expert e
+ *   is_token_in_rank       device uint8 [T,R]: 1 if some expert of t is on r
+ *   err                    device int32 [1]: status word (written by this call)
+ *   ws, ws_bytes           device workspace of ep_workspace_bytes(T,K,E,R)
+ * Any of the three outputs may be NULL to skip it.
+ */
+ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E,
+                                   int32_t R, int32_t* num_tokens_per_rank,
+                                   int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                                   int32_t* err, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dispatch (dispatch, comparative analysis sections 2.1-3.1): one received row
+ * per unmasked (t,k) ("expand" mode), rows ordered by (expert, source token, k)
+ * -- the deterministic order of section 8.4 -- each expert's segment padded to
+ * a multiple of A.  Padding rows hold zero bytes, scale 0, recv_topk_idx -1,
+ * weight 0 and metadata (-1,-1).
+ *   x                    device bf16 [T,H] (16-byte aligned rows)
+ *   topk_idx             device int64 [T,K]
+ *   topk_weights         device fp32 [T,K]
+ *   recv_x               device [recv_capacity, H]: bf16 (NONE) or 1-byte codes
+ *   recv_scales          device fp32 [recv_capacity, H/quant_size]; NULL for NONE
+ *   recv_topk_idx        device int32 [recv_capacity, K]: for the row of (t,k)
+ *                        with expert e on rank r, entry j is topk_idx[t,j] - r*L
+ *                        if that expert is on rank r, else -1
+ *   recv_topk_weights    device fp32 [recv_capacity, K]: topk_weights[t,j] where
+ *                        recv_topk_idx is >= 0, else 0
+ *   handle               caller-allocated arrays, see ep_handle_t; filled here
+ *   num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank: optional
+ *                        layout outputs as in ep_get_dispatch_layout (may be NULL)
+ *   ws, ws_bytes         device workspace of ep_workspace_bytes(T,K,E,R)
+ * The rows needed are psum_num_recv_tokens_per_expert[E-1]; if recv_capacity is
+ * smaller, *handle->err = EP_ERR_CAPACITY and no row at or past recv_capacity
+ * is written.
+ */
+ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                        const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                        const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                        int32_t* recv_topk_idx, float* recv_topk_weights,
+                        int64_t recv_capacity, ep_handle_t* handle,
+                        int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                        uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Combine (combine, comparative analysis section 9.2): for every token t
+ *   out[t] = bf16_rne( sum over k = 0..K-1 with dst_buffer_slot_idx[t,k] >= 0
+ *                      of topk_weights[t,k] * y[dst_buffer_slot_idx[t,k]] ),
+ * accumulated in fp32 with fused multiply-adds in k order from +0.
+ *   y              device bf16 [handle->recv_capacity, H]: expert outputs, in the
+ *                  received-row order of the dispatch that filled `handle`
+ *   handle         as filled by ep_dispatch (num_rounds is taken from it)
+ *   topk_weights   device fp32 [T,K]
+ *   out            device bf16 [T,H]
+ */
+ep_status_t ep_combine(const void* y, const ep_handle_t* handle, const float* topk_weights,
+                       void* out, void* stream);
+
+/* Waits for `stream`, then copies the device status word to *host_status.
+ * Returns EP_OK, or EP_ERR_CUDA if the wait or the copy failed. */
+ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status);
+
+/* The host copy a "do_cpu_sync" dispatch makes (comparative analysis,
+ * section 3.2): waits for `stream`, then copies the E unaligned per-expert
+ * counts to host_counts[E] (may be NULL) and the number of received rows
+ * (psum_num_recv_tokens_per_expert[E-1]) to *num_recv_rows (may be NULL). */
+ep_status_t ep_copy_recv_counts(const ep_handle_t* handle, void* stream, int32_t* host_counts,
+                                int64_t* num_recv_rows);
+
+/* A static string naming a status code. */
+const char* ep_status_string(ep_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_EP_H */

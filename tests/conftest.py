@@ -18,3 +18,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda", 0)
+
+
+def pytest_sessionstart(session):
+    # compile libep.so (sm_100a) and the C oracle if their sources are newer
+    from combine_topk_idx_rank_b200 import build as libbuild
+    from oracle import build as oracle_build
+    libbuild.build()
+    oracle_build.build()

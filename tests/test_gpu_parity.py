@@ -1,0 +1,230 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Sizes the oracle finishes in seconds that still span several 128-token chunks
+and a ragged last chunk, on every workload shape, seeds 0-2; plus the edge
+cases (no tokens, all entries masked, K=1, one expert per rank, minimum
+hidden, duplicate ids, group sizes 16..512, per-token FP8, power-of-two int8
+scales).  Bit-exact for layout, slots, metadata, rows, codes and scales;
+combine is bit-exact too and also meets the 1e-2 relative contract.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_topk_idx_rank_b200 import ep
+from combine_topk_idx_rank_b200.workloads import CONFIGS, make_workload, make_y
+
+from gpu_parity import (assert_combine_close, assert_layout_equal, assert_rows_equal, assert_slots_equal,
+                        gpu_dispatch, to_dev, u16)
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(name):
+    cfg = CONFIGS[name]
+    R = cfg.num_ranks
+    # a token count that is a multiple of R (and of the rounds) but not of 128
+    T = {"tiny": 256, "decode": 16 * 40, "prefill": 8 * 136, "qwen3": 16 * 40, "longseq": 8 * 8 * 17}[name]
+    H = {"tiny": 512, "decode": 1024, "prefill": 1536, "qwen3": 2048, "longseq": 1024}[name]
+    return cfg.scaled(num_tokens=T, hidden=H)
+
+
+def run_and_compare(cfg, seed, dev, num_rounds=None):
+    wl = make_workload(cfg, seed)
+    (recv_x, recv_scales, rti, rtw, h), lay, (x, ti, tw) = gpu_dispatch(cfg, wl, dev, num_rounds)
+    ref_lay = oracle.layout(wl.topk_idx, cfg.num_experts, cfg.num_ranks)
+    ref = oracle.dispatch(wl.x, wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks,
+                          cfg.expert_alignment, cfg.quant, cfg.quant_size, cfg.round_scale,
+                          cfg.num_rounds if num_rounds is None else num_rounds)
+    assert_layout_equal(lay, ref_lay)
+    assert_slots_equal(h, rti, rtw, ref)
+    assert_rows_equal(cfg, recv_x, recv_scales, ref["recv_x"], ref["recv_scales"])
+    # combine over expert outputs y (bf16, received-row order)
+    y_np = make_y(ref["num_recv_rows"], cfg.hidden, seed)
+    y = torch.from_numpy(y_np.view(np.int16)).view(torch.bfloat16).to(dev)
+    out = ep.ep_combine(y, h, tw)
+    torch.cuda.synchronize()
+    h.check()
+    ref_out = oracle.combine(y_np, ref["dst_buffer_slot_idx"], wl.topk_weights, cfg.num_ranks,
+                             cfg.num_rounds if num_rounds is None else num_rounds)
+    got = u16(out)
+    assert_combine_close(got, ref_out)
+    assert np.array_equal(got, ref_out)
+    return wl, ref, h
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_parity_small(name, seed, cuda_device):
+    run_and_compare(_small(name), seed, cuda_device)
+
+
+def test_identity_expert_round_trip(cuda_device):
+    cfg = _small("prefill")
+    wl = make_workload(cfg, 0)
+    (recv_x, _, _, _, h), _, (x, ti, tw) = gpu_dispatch(cfg, wl, cuda_device)
+    out = ep.ep_combine(recv_x.contiguous(), h, tw).float()
+    wsum = torch.where(ti >= 0, tw, torch.zeros_like(tw)).double().sum(1, keepdim=True)
+    ref = x.double() * wsum
+    assert torch.all((out.double() - ref).abs() <= 2.0 ** -8 * ref.abs() + 1e-30)
+
+
+def test_rounds_match_one_shot_on_gpu(cuda_device):
+    cfg = _small("longseq")
+    wl = make_workload(cfg, 1)
+    a, _, _ = gpu_dispatch(cfg, wl, cuda_device, num_rounds=1)
+    a = [t.clone() if t is not None else None for t in a[:4]]
+    b, _, _ = gpu_dispatch(cfg, wl, cuda_device, num_rounds=8)
+    for u, v in zip(a, b[:4]):
+        if u is not None:
+            assert torch.equal(u.view(torch.uint8), v.view(torch.uint8))
+
+
+def test_deterministic_repeat(cuda_device):
+    cfg = _small("qwen3")
+    wl = make_workload(cfg, 2)
+    a, _, _ = gpu_dispatch(cfg, wl, cuda_device)
+    a = [t.clone() for t in a[:4]]
+    b, _, _ = gpu_dispatch(cfg, wl, cuda_device)
+    for u, v in zip(a, b[:4]):
+        assert torch.equal(u.view(torch.uint8), v.view(torch.uint8))
+
+
+@pytest.mark.parametrize("quant,qs,rs", [("fp8", 16, False), ("fp8", 32, True), ("fp8", 64, False),
+                                         ("fp8", 256, True), ("fp8", 512, False), ("fp8", 1024, False),
+                                         ("fp8", 1024, True), ("int8", 128, False), ("int8", 128, True),
+                                         ("int8", 1024, True), ("int8", 512, False)])
+def test_quant_variants(quant, qs, rs, cuda_device):
+    cfg = CONFIGS["decode"].scaled(num_tokens=16 * 9, hidden=1024, quant=quant, quant_size=qs,
+                                   round_scale=rs, expert_alignment=4)
+    run_and_compare(cfg, 0, cuda_device)
+
+
+def test_edge_shapes(cuda_device):
+    base = CONFIGS["tiny"]
+    cases = [
+        base.scaled(num_tokens=8, num_topk=1),                               # K = 1
+        base.scaled(num_tokens=8 * 33, num_experts=8, num_topk=3),           # one expert per rank
+        base.scaled(num_tokens=8 * 20, hidden=8),                            # minimum hidden
+        base.scaled(num_tokens=8 * 50, hidden=8 * 7, expert_alignment=64),   # hidden not a power of 2
+        base.scaled(num_tokens=4 * 64, num_ranks=4, num_experts=1024, num_topk=16, hidden=64,
+                    expert_alignment=3),                                      # largest E and K
+        base.scaled(num_tokens=256 * 2, num_ranks=256, num_experts=256, num_topk=4, hidden=64),  # R = 256
+    ]
+    for cfg in cases:
+        run_and_compare(cfg, 0, cuda_device)
+
+
+def test_no_tokens(cuda_device):
+    cfg = CONFIGS["prefill"].scaled(num_tokens=0, hidden=256)
+    wl = make_workload(cfg, 0)
+    (recv_x, _, rti, rtw, h), lay, _ = gpu_dispatch(cfg, wl, cuda_device)
+    assert h.num_recv_rows == 0
+    assert torch.all(h.psum_num_recv_tokens_per_expert == 0)
+    assert torch.all(lay[0] == 0) and torch.all(lay[1] == 0)
+
+
+def test_all_masked_and_duplicates(cuda_device):
+    cfg = CONFIGS["tiny"].scaled(num_tokens=8 * 30, expert_alignment=4)
+    wl = make_workload(cfg, 0)
+    wl.topk_idx[:] = -1
+    wl.topk_weights[:] = 0
+    wl.topk_idx[3] = [5, 5]          # duplicate ids in one row: each (t, k) gets a row
+    wl.topk_weights[3] = [0.25, 0.75]
+    (recv_x, _, rti, rtw, h), lay, (x, ti, tw) = gpu_dispatch(cfg, wl, cuda_device)
+    ref = oracle.dispatch(wl.x, wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 4)
+    assert_slots_equal(h, rti, rtw, ref)
+    assert_rows_equal(cfg, recv_x, None, ref["recv_x"], None)
+    out = ep.ep_combine(recv_x.contiguous(), h, tw)
+    ref_out = oracle.combine_rows(ref["recv_x"], ref["dst_buffer_slot_idx"], wl.topk_weights)
+    assert np.array_equal(u16(out), ref_out)
+    assert np.all(ref_out[np.arange(ref_out.shape[0]) != 3] == 0)
+
+
+def test_e4m3_and_int8_conversion_exhaustive_over_bf16(cuda_device):
+    """Every bf16 value |v| <= 448 goes through the FP8 path with its group's
+    scale pinned to exactly 1 (each group holds 448), and every |v| <= 127
+    through the int8 path with scale 1 (each group holds 127)."""
+    for quant, top in (("fp8", 448.0), ("int8", 127.0)):
+        allv = (np.arange(0, 0x7f80, dtype=np.uint32) << 16).view(np.float32)
+        v = allv[allv <= top]
+        v = np.concatenate([v, -v]).astype(np.float32)
+        per = 127
+        ngroups = -(-v.size // per)
+        v = np.concatenate([v, np.zeros(ngroups * per - v.size, np.float32)]).reshape(ngroups, per)
+        g = np.concatenate([np.full((ngroups, 1), top, np.float32), v], axis=1)   # [ngroups, 128]
+        H = 1024
+        R = 8
+        T = -(-ngroups * 128 // H)
+        T = -(-T // R) * R
+        flat = np.zeros(T * H, np.float32)
+        flat[:g.size] = g.ravel()
+        flat[g.size:] = top
+        cfg = CONFIGS["tiny"].scaled(num_tokens=T, hidden=H, quant=quant, quant_size=128)
+        wl = make_workload(cfg, 0)
+        wl.x = torch.from_numpy(flat.reshape(T, H)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        (recv_x, recv_scales, rti, rtw, h), _, _ = gpu_dispatch(cfg, wl, cuda_device)
+        ref = oracle.dispatch(wl.x, wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 1,
+                              quant, 128, False)
+        assert np.all(ref["recv_scales"] == 1.0)
+        assert_rows_equal(cfg, recv_x, recv_scales, ref["recv_x"], ref["recv_scales"])
+
+
+def test_bad_expert_id_sets_status(cuda_device):
+    cfg = CONFIGS["tiny"]
+    wl = make_workload(cfg, 0)
+    wl.topk_idx[17, 1] = cfg.num_experts          # out of range
+    (recv_x, _, _, _, h), _, _ = gpu_dispatch(cfg, wl, cuda_device, do_cpu_sync=False)
+    torch.cuda.synchronize()
+    assert h.read_error() == ep.EP_ERR_BAD_EXPERT_ID
+    wl.topk_idx[17, 1] = -5
+    (_, _, _, _, h), _, _ = gpu_dispatch(cfg, wl, cuda_device, do_cpu_sync=False)
+    assert h.read_error() == ep.EP_ERR_BAD_EXPERT_ID
+    with pytest.raises(ep.EPError):
+        gpu_dispatch(cfg, wl, cuda_device, do_cpu_sync=True)
+    # the layout call reports it too
+    _, ti, _ = to_dev(wl, cuda_device)
+    with pytest.raises(ep.EPError) as e:
+        ep.ep_get_dispatch_layout(ti, cfg.num_experts, cfg.num_ranks)
+    assert e.value.status == ep.EP_ERR_BAD_EXPERT_ID
+
+
+def test_capacity_overflow_sets_status_and_writes_nothing_past_it(cuda_device):
+    cfg = CONFIGS["tiny"].scaled(expert_alignment=8)
+    wl = make_workload(cfg, 0)
+    ref = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 8)
+    need = ref["num_recv_rows"]
+    cap = need - 50
+    full = ep.alloc_dispatch_buffers(cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts,
+                                     cfg.num_ranks, 8, recv_capacity=need + 64, device=cuda_device)
+    for t in (full.recv_x, full.recv_topk_idx, full.recv_topk_weights, full.handle.recv_src_metadata):
+        t.view(torch.uint8).fill_(0xA5)
+    short = ep.DispatchBuffers(full.recv_x[:cap], None, full.recv_topk_idx[:cap], full.recv_topk_weights[:cap],
+                               full.handle, full.workspace, None, 128)
+    (_, _, _, _, h), _, _ = gpu_dispatch(cfg, wl, cuda_device, buffers=short, do_cpu_sync=False)
+    torch.cuda.synchronize()
+    assert h.read_error() == ep.EP_ERR_CAPACITY
+    for t in (full.recv_x, full.recv_topk_idx, full.recv_topk_weights, full.handle.recv_src_metadata):
+        assert torch.all(t[cap:].contiguous().view(torch.uint8) == 0xA5)
+
+
+def test_layout_call_matches_oracle(cuda_device):
+    for name in CONFIGS:
+        cfg = _small(name)
+        wl = make_workload(cfg, 5)
+        _, ti, _ = to_dev(wl, cuda_device)
+        got = ep.ep_get_dispatch_layout(ti, cfg.num_experts, cfg.num_ranks)
+        assert_layout_equal(got, oracle.layout(wl.topk_idx, cfg.num_experts, cfg.num_ranks))
+
+
+def test_cumulative_stats_accumulate(cuda_device):
+    cfg = _small("decode")
+    wl = make_workload(cfg, 0)
+    x, ti, tw = to_dev(wl, cuda_device)
+    stats = torch.zeros(cfg.num_experts, dtype=torch.int32, device=cuda_device)
+    for _ in range(3):
+        ep.ep_dispatch(x, ti, tw, 1, "fp8", num_experts=cfg.num_experts, num_ranks=cfg.num_ranks,
+                       cumulative_local_expert_recv_stats=stats, do_cpu_sync=False)
+    ref = oracle.layout(wl.topk_idx, cfg.num_experts, cfg.num_ranks)["num_tokens_per_expert"]
+    assert np.array_equal(stats.cpu().numpy(), 3 * ref)
