@@ -137,8 +137,10 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
         if (recv_scales == nullptr) return EP_ERR_INVALID_ARG;
     }
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
-        h->recv_src_metadata == nullptr || h->dst_buffer_slot_idx == nullptr || h->err == nullptr)
+        h->err == nullptr)
         return EP_ERR_INVALID_ARG;
+    if (T > 0 && h->dst_buffer_slot_idx == nullptr) return EP_ERR_INVALID_ARG;
+    if (recv_capacity > 0 && h->recv_src_metadata == nullptr) return EP_ERR_INVALID_ARG;
     if (recv_capacity > 0 && (recv_x == nullptr || recv_topk_idx == nullptr || recv_topk_weights == nullptr))
         return EP_ERR_INVALID_ARG;
     if (T > 0 && (x == nullptr || topk_idx == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
@@ -174,6 +176,21 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     s = cuda_status(launch_scan(sa, st));
     if (s) return s;
 
+    if (T > 0) {
+        SlotsArgs sl{};
+        sl.topk_idx = topk_idx; sl.topk_weights = topk_weights;
+        sl.T = T; sl.K = K; sl.E = E; sl.L = E / R;
+        sl.dst_slot = h->dst_buffer_slot_idx; sl.chunk_off = w.chunk_off;
+        sl.recv_meta = h->recv_src_metadata; sl.recv_topk_idx = recv_topk_idx;
+        sl.recv_topk_weights = recv_topk_weights;
+        sl.recv_scales = quant != EP_QUANT_NONE ? recv_scales : nullptr;
+        sl.nscales = quant != EP_QUANT_NONE ? H / quant_size : 0;
+        sl.capacity = recv_capacity;
+        sl.pad_base = w.pad_base; sl.pad_start = w.pad_start; sl.hdr = w.hdr;
+        sl.max_pad = E * (A - 1);
+        s = cuda_status(launch_slots(sl, st));
+        if (s) return s;
+    }
     if (opts->event_pack_begin) {
         s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
         if (s) return s;
@@ -183,16 +200,15 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
         for (int j = 0; j < rounds; ++j) {
             PackArgs pa{};
             pa.x = static_cast<const uint16_t*>(x);
-            pa.T = T; pa.H = H; pa.K = K; pa.E = E; pa.L = E / R;
-            pa.topk_idx = topk_idx; pa.topk_weights = topk_weights;
-            pa.dst_slot = h->dst_buffer_slot_idx; pa.chunk_off = w.chunk_off;
+            pa.H = H; pa.K = K; pa.E = E;
+            pa.dst_slot = h->dst_buffer_slot_idx;
             pa.recv_x = static_cast<uint8_t*>(recv_x); pa.recv_scales = recv_scales;
-            pa.recv_topk_idx = recv_topk_idx; pa.recv_topk_weights = recv_topk_weights;
-            pa.recv_meta = h->recv_src_metadata; pa.capacity = recv_capacity;
+            pa.capacity = recv_capacity;
             pa.pad_base = w.pad_base; pa.pad_start = w.pad_start; pa.hdr = w.hdr;
             pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
             pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
+            pa.err = h->err;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }
@@ -211,8 +227,9 @@ ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_we
     const int rounds = h->num_rounds;
     if (!sizes_ok(T, K, h->num_experts, R)) return EP_ERR_INVALID_ARG;
     if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
-    if (h->dst_buffer_slot_idx == nullptr || h->err == nullptr) return EP_ERR_INVALID_ARG;
-    if (T > 0 && (out == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
+    if (h->err == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (out == nullptr || topk_weights == nullptr || h->dst_buffer_slot_idx == nullptr))
+        return EP_ERR_INVALID_ARG;
     if (h->recv_capacity > 0 && y == nullptr) return EP_ERR_INVALID_ARG;
     if (!aligned16(y) || !aligned16(out)) return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;

@@ -4,8 +4,9 @@
 //   memset(ws counters) -> k_layout (one CTA per 128-token chunk: validated
 //   routing, per-chunk expert histograms, per-entry rank inside its chunk,
 //   is_token_in_rank, counters) -> k_scan (aligned expert segments, chunk
-//   offsets, padding map) -> k_pack per round (persistent: slots, metadata,
-//   row copy or fused quantisation, zeroed padding rows).
+//   offsets, padding map) -> k_slots (received row of every entry, per-row
+//   metadata) -> k_pack per round (persistent: TMA bulk row copies or fused
+//   quantisation, zeroed padding rows).
 // Combine is one persistent kernel per round: gather + k-order fp32 FMA.
 #pragma once
 
@@ -87,24 +88,37 @@ struct ScanArgs {
     int32_t* err_out;            // [1]
 };
 
-struct PackArgs {
-    const uint16_t* x;
-    int T, H, K, E, L;
+struct SlotsArgs {
     const int64_t* topk_idx;
     const float* topk_weights;
-    int32_t* dst_slot;          // in: rank inside chunk; out: received row
+    int T, K, E, L;
+    int32_t* dst_slot;          // in: rank inside chunk; out: received row (-1 = none)
     const int32_t* chunk_off;   // [nchunks,E] row offset of (chunk, expert)
-    uint8_t* recv_x;
-    float* recv_scales;
+    int32_t* recv_meta;
     int32_t* recv_topk_idx;
     float* recv_topk_weights;
-    int32_t* recv_meta;
+    float* recv_scales;         // null when not quantised
+    int nscales;                // scales per row (0 when not quantised)
+    int64_t capacity;
+    const int32_t* pad_base;
+    const int32_t* pad_start;
+    const int32_t* hdr;         // [2] = padding rows
+    int max_pad;                // host bound on padding rows: E * (A - 1)
+};
+
+struct PackArgs {
+    const uint16_t* x;
+    int H, K, E;
+    const int32_t* dst_slot;    // [T,K] received row of each entry (-1 = none)
+    uint8_t* recv_x;
+    float* recv_scales;
     int64_t capacity;
     const int32_t* pad_base;
     const int32_t* pad_start;
     const int32_t* hdr;         // [2] = padding rows
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
+    int32_t* err;
 };
 
 struct CombineArgs {
@@ -121,6 +135,7 @@ struct CombineArgs {
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_layout(const LayoutArgs& a, int nchunks, cudaStream_t st);
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
+cudaError_t launch_slots(const SlotsArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

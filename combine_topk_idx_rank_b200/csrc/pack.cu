@@ -1,93 +1,101 @@
 // Permute / pack: every source token's row is read from HBM once and written
-// to each of its received rows (one per unmasked top-k entry), as a bf16 bit
-// copy or quantised once per token on the fly:
+// to each of its received rows (one per unmasked top-k entry, rows already
+// resolved by k_slots into dst_buffer_slot_idx), as a bf16 bit copy or
+// quantised once per token on the fly:
 //   - FP8 e4m3 (OCP e4m3fn) or int8 with one fp32 scale per quant_size
 //     channels: scale = max(amax, 1e-4) / 448 (or / 127) by IEEE division,
 //     optionally rounded up to a power of two (round_scale / use_ue8m0 of
 //     low_latency_dispatch, "DeepEP communication library guide v2.1"),
 //     codes = RNE-saturating conversion of x / scale (IEEE division);
 //   - quant_size = 128 (group) or hidden (per token) (guide v2.1, 1.3.1).
-// The same persistent grid also zero-fills the padding rows that expert
-// alignment adds (comparative analysis, section 3.1), and writes the
-// per-row metadata (recv_src_metadata, recv_topk_idx, recv_topk_weights) and
-// the final dst_buffer_slot_idx.
+// The same persistent grid zero-fills the padding rows that expert alignment
+// adds (comparative analysis, section 3.1).
 //
-// Data movement: 16-byte vector loads that bypass L1 (x is read once) and
-// 16-byte stores; every row is a whole number of 16-byte vectors and, for
-// bf16 rows of 7168 channels, of 128-byte lines.
+// bf16 rows move entirely on the TMA engine: one warp per CTA runs an S-stage
+// ring in shared memory; lane 0 streams row chunks in with cp.async.bulk
+// (completion on an mbarrier) and, once a chunk has landed, issues one
+// cp.async.bulk store per destination row from the same shared-memory stage.
+// No register ever holds row data, and no multicast is used.
+// Quantised rows are computed by threads from 16-byte vector loads and
+// written with 16-byte vector stores.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
 #include "ep_internal.cuh"
 
+#ifndef EP_PACK_STAGES
+#define EP_PACK_STAGES 4
+#endif
+
 namespace ep {
 
 namespace {
 
-constexpr int kQuantNone = 0, kQuantFp8 = 1, kQuantInt8 = 2;
+constexpr int kQuantFp8 = 1, kQuantInt8 = 2;
+constexpr int kBulkChunk = 16384;          // max bytes per pipeline stage
+constexpr unsigned kSpinLimit = 1u << 24;  // bounded mbarrier waits
 
-struct ItemSmem {
-    int slot[kMaxTopk];
-    int e[kMaxTopk];
-    float w[kMaxTopk];
-    float red[33];
-};
-
-// Resolves the K received rows of token t, writes dst_buffer_slot_idx and the
-// per-row metadata.  Leaves the rows in s.slot (-1 = none).
-__device__ __forceinline__ void token_slots(const PackArgs& a, int t, ItemSmem& s) {
-    const int tid = threadIdx.x;
-    const int K = a.K;
-    if (tid < K) {
-        const int64_t v = a.topk_idx[(int64_t)t * K + tid];
-        const int e = (v >= 0 && v < a.E) ? (int)v : -1;
-        int slot = -1;
-        if (e >= 0) {
-            const int rank = a.dst_slot[(int64_t)t * K + tid];
-            const int64_t row = (int64_t)a.chunk_off[(size_t)(t / kChunkTokens) * a.E + e] + rank;
-            slot = (rank >= 0 && row < a.capacity) ? (int)row : -1;
-        }
-        a.dst_slot[(int64_t)t * K + tid] = slot;
-        s.slot[tid] = slot;
-        s.e[tid] = e;
-        s.w[tid] = a.topk_weights[(int64_t)t * K + tid];
-    }
-    __syncthreads();
-    if (tid < K) {
-        const int slot = s.slot[tid];
-        if (slot >= 0) {
-            const int rdst = s.e[tid] / a.L;
-            reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t, tid);
-            int32_t* ri = a.recv_topk_idx + (int64_t)slot * K;
-            float* rw = a.recv_topk_weights + (int64_t)slot * K;
-            for (int j = 0; j < K; ++j) {
-                const int ej = s.e[j];
-                const bool here = ej >= 0 && ej / a.L == rdst;
-                ri[j] = here ? ej - rdst * a.L : -1;
-                rw[j] = here ? s.w[j] : 0.0f;
-            }
-        }
-    }
+// ------------------------------------------------------ TMA bulk primitives
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for phase `parity` of `bar`; false if the bounded wait gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (unsigned n = 0; n < kSpinLimit; ++n)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Padding row number p (0-based over all experts) -> its row index.
 __device__ __forceinline__ int64_t pad_row(const PackArgs& a, const int* s_pad_base, int p) {
-    int lo = 0, hi = a.E;   // find the last e with pad_base[e] <= p
+    int lo = 0, hi = a.E;   // the last expert with pad_base <= p
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (s_pad_base[mid] <= p) lo = mid; else hi = mid;
     }
     return (int64_t)a.pad_start[lo] + (p - s_pad_base[lo]);
-}
-
-__device__ __forceinline__ void pad_metadata(const PackArgs& a, int64_t row, int nscales) {
-    const int tid = threadIdx.x;
-    if (tid == 0) reinterpret_cast<int2*>(a.recv_meta)[row] = make_int2(-1, -1);
-    for (int j = tid; j < a.K; j += blockDim.x) {
-        a.recv_topk_idx[row * a.K + j] = -1;
-        a.recv_topk_weights[row * a.K + j] = 0.0f;
-    }
-    for (int j = tid; j < nscales; j += blockDim.x) a.recv_scales[row * nscales + j] = 0.0f;
 }
 
 __device__ __forceinline__ float pow2_ceil_bits(float s) {
@@ -140,28 +148,161 @@ __device__ __forceinline__ float amax16(const float (&f)[16]) {
 }
 
 __device__ __forceinline__ float finish_scale(float amax, float qmax, int round_scale) {
-    float s = __fdiv_rn(fmaxf(amax, 1e-4f), qmax);
+    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), qmax);
     return round_scale ? pow2_ceil_bits(s) : s;
+}
+
+// Loads the K received rows of token t into s_slot (threads 0..K-1).
+__device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
+    if (threadIdx.x < a.K) s_slot[threadIdx.x] = a.dst_slot[(int64_t)t * a.K + threadIdx.x];
+}
+
+__device__ __forceinline__ void copy_pad_base(const PackArgs& a, int* s_pad_base) {
+    if (a.do_pad)
+        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
 }
 
 }  // namespace
 
-// ---------------------------------------------------------------- bf16 copy
+// ----------------------------------------------------- bf16: TMA bulk copy
+// Work unit = (token, chunk of its row); CTA b takes units b, b + grid, ...
+// Stage of the i-th own unit: i % S.  Lane 0 issues every bulk copy; lanes
+// 0..K-1 fetch the unit's destination rows one iteration ahead of use.
+template <int S>
+__global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* stage = smem;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * chunk_bytes);
+    int* sslot = reinterpret_cast<int*>(mbar + S);                 // [S][kMaxTopk]
+    int* s_pad_base = sslot + S * kMaxTopk;                          // [E+1]
+    const int lane = threadIdx.x;
+    const int K = a.K;
+    const int64_t row_bytes = (int64_t)a.H * 2;
+    const int nch = (int)((row_bytes + chunk_bytes - 1) / chunk_bytes);
+    const int n_units = a.n_tok_items * nch;
+    const int n_mine = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.x);
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
+        fence_mbar_init();
+    }
+    copy_pad_base(a, s_pad_base);
+    __syncwarp();
+
+    auto unit = [&](int j, int& t, int& c) {
+        const int u = (int)blockIdx.x + j * (int)gridDim.x;
+        const int item = u / nch;
+        c = u - item * nch;
+        t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
+    };
+    auto issue_load = [&](int j, int t, int c) {
+        const int64_t off = (int64_t)c * chunk_bytes;
+        const uint32_t bytes = (uint32_t)min((int64_t)chunk_bytes, row_bytes - off);
+        uint64_t* bar = &mbar[j % S];
+        mbar_expect_tx(bar, bytes);
+        bulk_load(stage + (size_t)(j % S) * chunk_bytes, xb + (int64_t)t * row_bytes + off, bytes, bar);
+    };
+
+    // prologue: units 0 .. S-2
+    const int pro = min(S - 1, n_mine);
+    for (int j = 0; j < pro; ++j) {
+        int t, c;
+        unit(j, t, c);
+        if (lane == 0) issue_load(j, t, c);
+        if (lane < K) sslot[(j % S) * kMaxTopk + lane] = a.dst_slot[(int64_t)t * K + lane];
+    }
+    __syncwarp();
+
+    bool ok = true;
+    int pending = -1;
+    int i = 0;
+    for (; i < n_mine; ++i) {
+        const int s = i % S;
+        // slots fetched last iteration belong to unit i + S - 2
+        if (i >= 1 && i + S - 2 < n_mine && lane < K) sslot[((i + S - 2) % S) * kMaxTopk + lane] = pending;
+        // lane 0 waits for the stage; the verdict is broadcast so the warp stays converged
+        int landed = lane == 0 ? (int)mbar_wait(&mbar[s], (uint32_t)((i / S) & 1)) : 0;
+        landed = __shfl_sync(0xffffffffu, landed, 0);
+        if (!landed) {
+            ok = false;
+            break;
+        }
+        int t, c;
+        unit(i, t, c);
+        if (lane == 0) {
+            const int64_t off = (int64_t)c * chunk_bytes;
+            const uint32_t bytes = (uint32_t)min((int64_t)chunk_bytes, row_bytes - off);
+            fence_proxy_async_smem();
+            for (int k = 0; k < K; ++k) {
+                const int slot = sslot[s * kMaxTopk + k];
+                if (slot >= 0) bulk_store(a.recv_x + (int64_t)slot * row_bytes + off, stage + (size_t)s * chunk_bytes, bytes);
+            }
+            bulk_commit();
+            bulk_wait_read<1>();   // the stores of unit i-1 have read their stage
+        }
+        __syncwarp();
+        const int nxt = i + S - 1;
+        if (nxt < n_mine) {
+            int tn, cn;
+            unit(nxt, tn, cn);
+            if (lane == 0) issue_load(nxt, tn, cn);
+            if (lane < K) pending = a.dst_slot[(int64_t)tn * K + lane];
+        }
+    }
+    if (!ok) {
+        set_error(a.err, EP_ERR_TIMEOUT);
+        // let every load still in flight land before the CTA releases its smem
+        if (lane == 0) {
+            for (int j = i; j < min(n_mine, i + S - 1); ++j) mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1));
+            bulk_wait_all();
+        }
+        __syncwarp();
+        return;
+    }
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+
+    // padding rows: bulk stores from a zeroed stage
+    const int n_pad = a.do_pad ? a.hdr[2] : 0;
+    const int pad_units = n_pad * nch;
+    if ((int)blockIdx.x < pad_units) {
+        for (int b = lane * 16; b < chunk_bytes; b += 32 * 16)
+            *reinterpret_cast<uint4*>(stage + b) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            for (int u = blockIdx.x; u < pad_units; u += gridDim.x) {
+                const int p = u / nch, c = u - p * nch;
+                const int64_t row = pad_row(a, s_pad_base, p);
+                const int64_t off = (int64_t)c * chunk_bytes;
+                const uint32_t bytes = (uint32_t)min((int64_t)chunk_bytes, row_bytes - off);
+                if (row < a.capacity) bulk_store(a.recv_x + row * row_bytes + off, stage, bytes);
+            }
+            bulk_commit();
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+// ----------------------------------------------- bf16: vector loads/stores
+// Alternative data path (16-byte ld/st through registers), kept for
+// comparison with the bulk-copy path.
 template <int VPT>
 __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
-    __shared__ ItemSmem s;
+    __shared__ int s_slot[kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1];
     const int tid = threadIdx.x;
     const int V = a.H / 8;   // 16-byte vectors per row
     const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    if (a.do_pad)
-        for (int i = tid; i <= a.E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
+    copy_pad_base(a, s_pad_base);
     __syncthreads();
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
             const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
-            token_slots(a, t, s);
+            load_slots(a, t, s_slot);
+            __syncthreads();
             const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
             for (int v0 = 0; v0 < V; v0 += VPT * blockDim.x) {
                 uint4 r[VPT];
@@ -171,7 +312,7 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
                     if (v < V) r[u] = ld_nc_v4(xr + v);
                 }
                 for (int k = 0; k < a.K; ++k) {
-                    const int slot = s.slot[k];
+                    const int slot = s_slot[k];
                     if (slot < 0) continue;
                     uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)slot * a.H * 2);
 #pragma unroll
@@ -186,7 +327,6 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H * 2);
                 for (int v = tid; v < V; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                pad_metadata(a, row, 0);
             }
         }
         __syncthreads();
@@ -198,7 +338,7 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 // store); a group of G channels is G/16 adjacent lanes, reduced by shuffles.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
-    __shared__ ItemSmem s;
+    __shared__ int s_slot[kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1];
     constexpr int kLanes = G / 16;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
@@ -206,14 +346,14 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
     const int U = a.H / 16;
     const int nscales = a.H / G;
     const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    if (a.do_pad)
-        for (int i = tid; i <= a.E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
+    copy_pad_base(a, s_pad_base);
     __syncthreads();
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
             const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
-            token_slots(a, t, s);
+            load_slots(a, t, s_slot);
+            __syncthreads();
             const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
             for (int u0 = 0; u0 < U; u0 += UPT * blockDim.x) {
                 uint4 q[UPT];
@@ -235,7 +375,7 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
                     q[j] = quant16<QUANT>(f, sc[j]);
                 }
                 for (int k = 0; k < a.K; ++k) {
-                    const int slot = s.slot[k];
+                    const int slot = s_slot[k];
                     if (slot < 0) continue;
                     uint8_t* dst = a.recv_x + (size_t)slot * a.H;
 #pragma unroll
@@ -253,7 +393,6 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                pad_metadata(a, row, nscales);
             }
         }
         __syncthreads();
@@ -265,21 +404,21 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
 // the block reduces its amax.
 template <int QUANT, int UPT>
 __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
-    __shared__ ItemSmem s;
+    __shared__ int s_slot[kMaxTopk];
+    __shared__ float s_red[33];
     __shared__ int s_pad_base[kMaxExperts + 1];
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarps = blockDim.x >> 5;
     const int U = a.H / 16;
     const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    if (a.do_pad)
-        for (int i = tid; i <= a.E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
+    copy_pad_base(a, s_pad_base);
     __syncthreads();
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
             const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
-            token_slots(a, t, s);
+            load_slots(a, t, s_slot);
             const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
             uint4 raw[UPT][2];
 #pragma unroll
@@ -301,31 +440,28 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) s.red[warp] = m;
+            if (lane == 0) s_red[warp] = m;
             __syncthreads();
             if (warp == 0) {
-                float v = lane < nwarps ? s.red[lane] : 0.0f;
+                float v = lane < nwarps ? s_red[lane] : 0.0f;
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                if (lane == 0) s.red[32] = v;
+                if (lane == 0) s_red[32] = v;
             }
             __syncthreads();
-            const float sc = finish_scale(s.red[32], kQmax, a.round_scale);
-            uint4 q[UPT];
-#pragma unroll
-            for (int j = 0; j < UPT; ++j) {
-                float f[16];
-                unpack16(raw[j][0], raw[j][1], f);
-                q[j] = quant16<QUANT>(f, sc);
-            }
+            const float sc = finish_scale(s_red[32], kQmax, a.round_scale);
             for (int k = 0; k < a.K; ++k) {
-                const int slot = s.slot[k];
+                const int slot = s_slot[k];
                 if (slot < 0) continue;
                 uint8_t* dst = a.recv_x + (size_t)slot * a.H;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
                     const int u = j * blockDim.x + tid;
-                    if (u < U) st_v4(dst + 16 * (size_t)u, q[j]);
+                    if (u < U) {
+                        float f[16];
+                        unpack16(raw[j][0], raw[j][1], f);
+                        st_v4(dst + 16 * (size_t)u, quant16<QUANT>(f, sc));
+                    }
                 }
                 if (tid == 0) a.recv_scales[slot] = sc;
             }
@@ -334,7 +470,6 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                pad_metadata(a, row, 1);
             }
         }
         __syncthreads();
@@ -345,9 +480,9 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
 namespace {
 
 template <typename Kern>
-int blocks_per_sm(Kern k, int threads) {
+int blocks_per_sm(Kern k, int threads, size_t smem) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, 0) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 1) n = 1;
     return n;
 }
 
@@ -355,7 +490,7 @@ inline int round_up32(int x) { return (x + 31) & ~31; }
 
 template <typename Kern>
 cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
-    const int grid = device_sm_count() * blocks_per_sm(k, threads);
+    const int grid = device_sm_count() * blocks_per_sm(k, threads, 0);
     k<<<grid, threads, 0, st>>>(a);
     return cudaGetLastError();
 }
@@ -386,15 +521,33 @@ cudaError_t launch_token(const PackArgs& a, cudaStream_t st) {
     return run(k_pack_token<QUANT, 4>, threads, a, st);
 }
 
+cudaError_t launch_bulk(const PackArgs& a, cudaStream_t st) {
+    constexpr int S = EP_PACK_STAGES;
+    const int64_t row_bytes = (int64_t)a.H * 2;
+    // equal chunks of at most kBulkChunk bytes, each a multiple of 16
+    const int nch = (int)((row_bytes + kBulkChunk - 1) / kBulkChunk);
+    const int chunk = (int)(((row_bytes + nch - 1) / nch + 15) / 16 * 16);
+    const size_t smem = (size_t)S * chunk + S * sizeof(uint64_t) + S * kMaxTopk * sizeof(int) +
+                        (kMaxExperts + 1) * sizeof(int);
+    cudaError_t e = cudaFuncSetAttribute(k_pack_bulk<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = device_sm_count() * blocks_per_sm(k_pack_bulk<S>, 32, smem);
+    k_pack_bulk<S><<<grid, 32, smem, st>>>(a, chunk);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st) {
     if (quant == EP_QUANT_NONE) {
+#ifdef EP_PACK_VECTOR
         const int V = a.H / 8;
-        // threads: a multiple of 32 that splits the row into passes of 4 vectors
         const int passes = (V + 4 * 256 - 1) / (4 * 256);
         const int threads = min(256, round_up32((V + 4 * passes - 1) / (4 * passes)));
         return run(k_pack_bf16<4>, threads, a, st);
+#else
+        return launch_bulk(a, st);
+#endif
     }
     const bool per_token = a.quant_size == a.H;
     if (quant == EP_QUANT_FP8_E4M3)

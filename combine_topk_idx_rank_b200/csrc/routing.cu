@@ -219,6 +219,78 @@ __global__ void __launch_bounds__(1024) k_scan(ScanArgs a) {
     }
 }
 
+// Turns every entry's rank inside its chunk into its received row,
+// row = offset[chunk][e] + rank, writes dst_buffer_slot_idx and the per-row
+// metadata of the receiving side: recv_src_metadata = (t, k), and for
+// recv_topk_idx / recv_topk_weights the token's top-k entries whose experts
+// live on the receiving rank (local ids), -1 / 0 elsewhere.  The threads past
+// the T*K entries fill the padding rows' metadata: (-1, -1), -1, 0, scale 0.
+__global__ void __launch_bounds__(256) k_slots(SlotsArgs a) {
+    __shared__ int s_pad_base[kMaxExperts + 1];
+    const int K = a.K, E = a.E;
+    const int64_t n_ent = (int64_t)a.T * K;
+    const int n_pad = a.hdr[2];
+    if (a.max_pad > 0)
+        for (int i = threadIdx.x; i <= E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
+    __syncthreads();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_ent + a.max_pad; i += stride) {
+        if (i < n_ent) {
+            const int t = (int)(i / K), k = (int)(i - (int64_t)t * K);
+            const int64_t v = a.topk_idx[i];
+            const int e = (v >= 0 && v < E) ? (int)v : -1;
+            int slot = -1;
+            if (e >= 0) {
+                const int rank = a.dst_slot[i];
+                const int64_t row = (int64_t)a.chunk_off[(size_t)(t / kChunkTokens) * E + e] + rank;
+                slot = (rank >= 0 && row < a.capacity) ? (int)row : -1;
+            }
+            a.dst_slot[i] = slot;
+            if (slot >= 0) {
+                reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t, k);
+                const int rdst = e / a.L;
+                const int64_t* row_ids = a.topk_idx + (int64_t)t * K;
+                const float* row_w = a.topk_weights + (int64_t)t * K;
+                int32_t* ri = a.recv_topk_idx + (int64_t)slot * K;
+                float* rw = a.recv_topk_weights + (int64_t)slot * K;
+                for (int j = 0; j < K; ++j) {
+                    const int64_t ej = __ldg(row_ids + j);
+                    const bool here = ej >= 0 && ej < E && (int)ej / a.L == rdst;
+                    ri[j] = here ? (int)ej - rdst * a.L : -1;
+                    rw[j] = here ? __ldg(row_w + j) : 0.0f;
+                }
+            }
+        } else {
+            const int p = (int)(i - n_ent);
+            if (p < n_pad) {
+                int lo = 0, hi = E;   // last expert with pad_base <= p
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_pad_base[mid] <= p) lo = mid; else hi = mid;
+                }
+                const int64_t row = (int64_t)a.pad_start[lo] + (p - s_pad_base[lo]);
+                if (row < a.capacity) {
+                    reinterpret_cast<int2*>(a.recv_meta)[row] = make_int2(-1, -1);
+                    for (int j = 0; j < K; ++j) {
+                        a.recv_topk_idx[row * K + j] = -1;
+                        a.recv_topk_weights[row * K + j] = 0.0f;
+                    }
+                    for (int j = 0; j < a.nscales; ++j) a.recv_scales[row * a.nscales + j] = 0.0f;
+                }
+            }
+        }
+    }
+}
+
+cudaError_t launch_slots(const SlotsArgs& a, cudaStream_t st) {
+    const int64_t work = (int64_t)a.T * a.K + a.max_pad;
+    if (work <= 0) return cudaSuccess;
+    const int64_t blocks = (work + 255) / 256;
+    const int grid = (int)(blocks < (int64_t)device_sm_count() * 8 ? blocks : (int64_t)device_sm_count() * 8);
+    k_slots<<<grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_layout(const LayoutArgs& a, int nchunks, cudaStream_t st) {
     const size_t smem = sizeof(int32_t) * (kLayoutWarps * a.E + kChunkTokens * a.K + a.R) +
                         (size_t)kChunkTokens * a.R;

@@ -57,11 +57,11 @@ class _Handle(C.Structure):
                 ("dst_buffer_slot_idx", C.c_void_p), ("err", C.c_void_p)]
 
 
-def _load():
-    if not os.path.exists(_LIB_PATH):
-        raise ImportError(f"libep.so not found at {_LIB_PATH}; build it with "
+def _load(path: str = _LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(f"libep.so not found at {path}; build it with "
                           "`python -m combine_topk_idx_rank_b200.build`")
-    L = C.CDLL(_LIB_PATH)
+    L = C.CDLL(path)
     p, i32, i64, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
     L.ep_recv_capacity_bound.argtypes = [i32, i32, i32, i32]
     L.ep_recv_capacity_bound.restype = i64

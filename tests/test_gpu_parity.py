@@ -111,6 +111,9 @@ def test_edge_shapes(cuda_device):
         base.scaled(num_tokens=4 * 64, num_ranks=4, num_experts=1024, num_topk=16, hidden=64,
                     expert_alignment=3),                                      # largest E and K
         base.scaled(num_tokens=256 * 2, num_ranks=256, num_experts=256, num_topk=4, hidden=64),  # R = 256
+        base.scaled(num_tokens=8 * 12, hidden=12000, expert_alignment=5),    # rows of 2 bulk chunks
+        base.scaled(num_tokens=8 * 6, hidden=20008),                          # 3 unequal bulk chunks
+        base.scaled(num_tokens=8 * 2, hidden=65536, num_topk=3),              # largest hidden
     ]
     for cfg in cases:
         run_and_compare(cfg, 0, cuda_device)
