@@ -17,6 +17,8 @@ namespace ep {
 
 template <int KMAX, int VPT>
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+    grid_dependency_wait();
+    grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     __shared__ int s_n;
@@ -107,8 +109,7 @@ cudaError_t run(Kern k, int threads, const CombineArgs& a, cudaStream_t st) {
         per_sm = 1;
     const int grid = min(a.n_items, device_sm_count() * per_sm);
     if (grid <= 0) return cudaSuccess;
-    k<<<grid, threads, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(k, dim3(grid), dim3(threads), 0, st, a);
 }
 
 }  // namespace

@@ -39,18 +39,19 @@ ep_status_t cuda_status(cudaError_t e) {
 
 struct WsPtrs {
     int32_t* hdr;
-    int32_t* counts;
-    int32_t* rank_counts;
     int32_t* pad_base;
     int32_t* pad_start;
+    int32_t* chunk_hist;
     int32_t* chunk_off;
+    int32_t* chunk_rcnt;
+    int32_t* chunk_err;
 };
 
 WsPtrs carve(void* ws, const WsLayout& L) {
     char* b = static_cast<char*>(ws);
-    return WsPtrs{reinterpret_cast<int32_t*>(b + L.hdr), reinterpret_cast<int32_t*>(b + L.counts),
-                  reinterpret_cast<int32_t*>(b + L.rank_counts), reinterpret_cast<int32_t*>(b + L.pad_base),
-                  reinterpret_cast<int32_t*>(b + L.pad_start), reinterpret_cast<int32_t*>(b + L.chunk_off)};
+    auto at = [&](size_t off) { return reinterpret_cast<int32_t*>(b + off); };
+    return WsPtrs{at(L.hdr), at(L.pad_base), at(L.pad_start), at(L.chunk_hist),
+                  at(L.chunk_off), at(L.chunk_rcnt), at(L.chunk_err)};
 }
 
 }  // namespace
@@ -92,18 +93,17 @@ ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K
     if (ws_bytes < L.total) return EP_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const WsPtrs w = carve(ws, L);
-    ep_status_t s = cuda_status(cudaMemsetAsync(ws, 0, L.zero_bytes, st));
-    if (s) return s;
+    ep_status_t s;
     if (T > 0) {
-        LayoutArgs la{topk_idx, T, K, E, R, E / R, nullptr, nullptr, is_token_in_rank, nullptr,
-                      w.counts, w.rank_counts, w.hdr};
+        LayoutArgs la{topk_idx, T, K, E, R, E / R, L.log2_chunk, nullptr, w.chunk_hist, is_token_in_rank,
+                      nullptr, w.chunk_rcnt, w.chunk_err};
         s = cuda_status(launch_layout(la, L.nchunks, st));
         if (s) return s;
     }
     ScanArgs sa{};
     sa.E = E; sa.R = R; sa.A = 1; sa.nchunks = L.nchunks;
     sa.capacity = 0; sa.check_capacity = 0;
-    sa.counts = w.counts; sa.rank_counts = w.rank_counts; sa.layout_err = w.hdr;
+    sa.chunk_hist = w.chunk_hist; sa.chunk_rcnt = w.chunk_rcnt; sa.chunk_err = w.chunk_err;
     sa.chunk_off = nullptr; sa.pad_base = nullptr; sa.pad_start = nullptr; sa.hdr = w.hdr;
     sa.num_tokens_per_expert = num_tokens_per_expert;
     sa.num_tokens_per_rank = num_tokens_per_rank;
@@ -153,18 +153,17 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
     h->hidden = H; h->expert_alignment = A; h->num_rounds = rounds; h->recv_capacity = recv_capacity;
 
-    ep_status_t s = cuda_status(cudaMemsetAsync(ws, 0, L.zero_bytes, st));
-    if (s) return s;
+    ep_status_t s;
     if (T > 0) {
-        LayoutArgs la{topk_idx, T, K, E, R, E / R, h->dst_buffer_slot_idx, w.chunk_off,
-                      is_token_in_rank, h->topk_idx, w.counts, w.rank_counts, w.hdr};
+        LayoutArgs la{topk_idx, T, K, E, R, E / R, L.log2_chunk, h->dst_buffer_slot_idx, w.chunk_hist,
+                      is_token_in_rank, h->topk_idx, w.chunk_rcnt, w.chunk_err};
         s = cuda_status(launch_layout(la, L.nchunks, st));
         if (s) return s;
     }
     ScanArgs sa{};
     sa.E = E; sa.R = R; sa.A = A; sa.nchunks = L.nchunks;
     sa.capacity = recv_capacity; sa.check_capacity = 1;
-    sa.counts = w.counts; sa.rank_counts = w.rank_counts; sa.layout_err = w.hdr;
+    sa.chunk_hist = w.chunk_hist; sa.chunk_rcnt = w.chunk_rcnt; sa.chunk_err = w.chunk_err;
     sa.chunk_off = T > 0 ? w.chunk_off : nullptr;
     sa.pad_base = w.pad_base; sa.pad_start = w.pad_start; sa.hdr = w.hdr;
     sa.psum = h->psum_num_recv_tokens_per_expert;
@@ -179,7 +178,9 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     if (T > 0) {
         SlotsArgs sl{};
         sl.topk_idx = topk_idx; sl.topk_weights = topk_weights;
-        sl.T = T; sl.K = K; sl.E = E; sl.L = E / R;
+        sl.T = T; sl.K = K; sl.E = E; sl.L = E / R; sl.log2_chunk = L.log2_chunk;
+        sl.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
+                       aligned16(recv_topk_weights);
         sl.dst_slot = h->dst_buffer_slot_idx; sl.chunk_off = w.chunk_off;
         sl.recv_meta = h->recv_src_metadata; sl.recv_topk_idx = recv_topk_idx;
         sl.recv_topk_weights = recv_topk_weights;

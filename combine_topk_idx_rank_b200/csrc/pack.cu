@@ -170,6 +170,8 @@ __device__ __forceinline__ void copy_pad_base(const PackArgs& a, int* s_pad_base
 // 0..K-1 fetch the unit's destination rows one iteration ahead of use.
 template <int S>
 __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
+    grid_dependency_wait();
+    grid_launch_dependents();
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* stage = smem;
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * chunk_bytes);
@@ -290,6 +292,8 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
 // comparison with the bulk-copy path.
 template <int VPT>
 __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
+    grid_dependency_wait();
+    grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1];
     const int tid = threadIdx.x;
@@ -338,6 +342,8 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 // store); a group of G channels is G/16 adjacent lanes, reduced by shuffles.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
+    grid_dependency_wait();
+    grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1];
     constexpr int kLanes = G / 16;
@@ -404,6 +410,8 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
 // the block reduces its amax.
 template <int QUANT, int UPT>
 __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
+    grid_dependency_wait();
+    grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
     __shared__ float s_red[33];
     __shared__ int s_pad_base[kMaxExperts + 1];
@@ -450,6 +458,13 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             }
             __syncthreads();
             const float sc = finish_scale(s_red[32], kQmax, a.round_scale);
+            // quantise once; raw[j][0] is reused to hold the 16 codes of unit j
+#pragma unroll
+            for (int j = 0; j < UPT; ++j) {
+                float f[16];
+                unpack16(raw[j][0], raw[j][1], f);
+                raw[j][0] = quant16<QUANT>(f, sc);
+            }
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[k];
                 if (slot < 0) continue;
@@ -457,11 +472,7 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
                     const int u = j * blockDim.x + tid;
-                    if (u < U) {
-                        float f[16];
-                        unpack16(raw[j][0], raw[j][1], f);
-                        st_v4(dst + 16 * (size_t)u, quant16<QUANT>(f, sc));
-                    }
+                    if (u < U) st_v4(dst + 16 * (size_t)u, raw[j][0]);
                 }
                 if (tid == 0) a.recv_scales[slot] = sc;
             }
@@ -491,8 +502,7 @@ inline int round_up32(int x) { return (x + 31) & ~31; }
 template <typename Kern>
 cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
     const int grid = device_sm_count() * blocks_per_sm(k, threads, 0);
-    k<<<grid, threads, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(k, dim3(grid), dim3(threads), 0, st, a);
 }
 
 template <int QUANT>
@@ -532,8 +542,7 @@ cudaError_t launch_bulk(const PackArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k_pack_bulk<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = device_sm_count() * blocks_per_sm(k_pack_bulk<S>, 32, smem);
-    k_pack_bulk<S><<<grid, 32, smem, st>>>(a, chunk);
-    return cudaGetLastError();
+    return launch_dependent(k_pack_bulk<S>, dim3(grid), dim3(32), smem, st, a, chunk);
 }
 
 }  // namespace
