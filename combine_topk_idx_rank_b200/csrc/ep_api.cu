@@ -37,21 +37,26 @@ ep_status_t cuda_status(cudaError_t e) {
     return EP_ERR_CUDA;
 }
 
-struct WsPtrs {
-    int32_t* hdr;
-    int32_t* pad_base;
-    int32_t* pad_start;
-    int32_t* chunk_hist;
-    int32_t* chunk_off;
-    int32_t* chunk_rcnt;
-    int32_t* chunk_err;
-};
-
-WsPtrs carve(void* ws, const WsLayout& L) {
+// Routing arguments common to the layout call and dispatch.
+RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const float* topk_weights,
+                     int T, int K, int E, int R) {
     char* b = static_cast<char*>(ws);
     auto at = [&](size_t off) { return reinterpret_cast<int32_t*>(b + off); };
-    return WsPtrs{at(L.hdr), at(L.pad_base), at(L.pad_start), at(L.chunk_hist),
-                  at(L.chunk_off), at(L.chunk_rcnt), at(L.chunk_err)};
+    RouteArgs r{};
+    r.topk_idx = topk_idx;
+    r.topk_weights = topk_weights;
+    r.T = T; r.K = K; r.E = E; r.R = R; r.L = E / R; r.A = 1;
+    r.log2_chunk = L.log2_chunk;
+    r.nchunks = L.nchunks;
+    r.barrier = reinterpret_cast<unsigned*>(at(L.hdr));
+    r.hdr = at(L.hdr);
+    r.pad_base = at(L.pad_base);
+    r.pad_start = at(L.pad_start);
+    r.col_total = at(L.col_total);
+    r.chunk_hist = at(L.chunk_hist);
+    r.chunk_rcnt = at(L.chunk_rcnt);
+    r.chunk_err = at(L.chunk_err);
+    return r;
 }
 
 }  // namespace
@@ -91,24 +96,13 @@ ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K
     if (T > 0 && topk_idx == nullptr) return EP_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(T, K, E, R);
     if (ws_bytes < L.total) return EP_ERR_INVALID_ARG;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WsPtrs w = carve(ws, L);
-    ep_status_t s;
-    if (T > 0) {
-        LayoutArgs la{topk_idx, T, K, E, R, E / R, L.log2_chunk, nullptr, w.chunk_hist, is_token_in_rank,
-                      nullptr, w.chunk_rcnt, w.chunk_err};
-        s = cuda_status(launch_layout(la, L.nchunks, st));
-        if (s) return s;
-    }
-    ScanArgs sa{};
-    sa.E = E; sa.R = R; sa.A = 1; sa.nchunks = L.nchunks;
-    sa.capacity = 0; sa.check_capacity = 0;
-    sa.chunk_hist = w.chunk_hist; sa.chunk_rcnt = w.chunk_rcnt; sa.chunk_err = w.chunk_err;
-    sa.chunk_off = nullptr; sa.pad_base = nullptr; sa.pad_start = nullptr; sa.hdr = w.hdr;
-    sa.num_tokens_per_expert = num_tokens_per_expert;
-    sa.num_tokens_per_rank = num_tokens_per_rank;
-    sa.err_out = err;
-    return cuda_status(launch_scan(sa, st));
+    RouteArgs r = route_args(ws, L, topk_idx, nullptr, T, K, E, R);
+    r.assign = 0;
+    r.is_token_in_rank = is_token_in_rank;
+    r.num_tokens_per_expert = num_tokens_per_expert;
+    r.num_tokens_per_rank = num_tokens_per_rank;
+    r.err_out = err;
+    return cuda_status(launch_route(r, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
@@ -149,49 +143,32 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     if (ws == nullptr || ws_bytes < L.total) return EP_ERR_INVALID_ARG;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WsPtrs w = carve(ws, L);
     h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
     h->hidden = H; h->expert_alignment = A; h->num_rounds = rounds; h->recv_capacity = recv_capacity;
 
-    ep_status_t s;
-    if (T > 0) {
-        LayoutArgs la{topk_idx, T, K, E, R, E / R, L.log2_chunk, h->dst_buffer_slot_idx, w.chunk_hist,
-                      is_token_in_rank, h->topk_idx, w.chunk_rcnt, w.chunk_err};
-        s = cuda_status(launch_layout(la, L.nchunks, st));
-        if (s) return s;
-    }
-    ScanArgs sa{};
-    sa.E = E; sa.R = R; sa.A = A; sa.nchunks = L.nchunks;
-    sa.capacity = recv_capacity; sa.check_capacity = 1;
-    sa.chunk_hist = w.chunk_hist; sa.chunk_rcnt = w.chunk_rcnt; sa.chunk_err = w.chunk_err;
-    sa.chunk_off = T > 0 ? w.chunk_off : nullptr;
-    sa.pad_base = w.pad_base; sa.pad_start = w.pad_start; sa.hdr = w.hdr;
-    sa.psum = h->psum_num_recv_tokens_per_expert;
-    sa.num_recv = h->num_recv_tokens_per_expert;
-    sa.num_tokens_per_expert = num_tokens_per_expert;
-    sa.num_tokens_per_rank = num_tokens_per_rank;
-    sa.cumulative = opts->cumulative_local_expert_recv_stats;
-    sa.err_out = h->err;
-    s = cuda_status(launch_scan(sa, st));
+    RouteArgs r = route_args(ws, L, topk_idx, topk_weights, T, K, E, R);
+    r.A = A;
+    r.capacity = recv_capacity;
+    r.check_capacity = 1;
+    r.assign = 1;
+    r.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
+                  aligned16(recv_topk_weights);
+    r.nscales = quant != EP_QUANT_NONE ? H / quant_size : 0;
+    r.dst_slot = h->dst_buffer_slot_idx;
+    r.topk_copy = h->topk_idx;
+    r.recv_meta = h->recv_src_metadata;
+    r.recv_topk_idx = recv_topk_idx;
+    r.recv_topk_weights = recv_topk_weights;
+    r.recv_scales = quant != EP_QUANT_NONE ? recv_scales : nullptr;
+    r.is_token_in_rank = is_token_in_rank;
+    r.psum = h->psum_num_recv_tokens_per_expert;
+    r.num_recv = h->num_recv_tokens_per_expert;
+    r.num_tokens_per_expert = num_tokens_per_expert;
+    r.num_tokens_per_rank = num_tokens_per_rank;
+    r.cumulative = opts->cumulative_local_expert_recv_stats;
+    r.err_out = h->err;
+    ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-
-    if (T > 0) {
-        SlotsArgs sl{};
-        sl.topk_idx = topk_idx; sl.topk_weights = topk_weights;
-        sl.T = T; sl.K = K; sl.E = E; sl.L = E / R; sl.log2_chunk = L.log2_chunk;
-        sl.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
-                       aligned16(recv_topk_weights);
-        sl.dst_slot = h->dst_buffer_slot_idx; sl.chunk_off = w.chunk_off;
-        sl.recv_meta = h->recv_src_metadata; sl.recv_topk_idx = recv_topk_idx;
-        sl.recv_topk_weights = recv_topk_weights;
-        sl.recv_scales = quant != EP_QUANT_NONE ? recv_scales : nullptr;
-        sl.nscales = quant != EP_QUANT_NONE ? H / quant_size : 0;
-        sl.capacity = recv_capacity;
-        sl.pad_base = w.pad_base; sl.pad_start = w.pad_start; sl.hdr = w.hdr;
-        sl.max_pad = E * (A - 1);
-        s = cuda_status(launch_slots(sl, st));
-        if (s) return s;
-    }
     if (opts->event_pack_begin) {
         s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
         if (s) return s;
@@ -205,7 +182,7 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
             pa.dst_slot = h->dst_buffer_slot_idx;
             pa.recv_x = static_cast<uint8_t*>(recv_x); pa.recv_scales = recv_scales;
             pa.capacity = recv_capacity;
-            pa.pad_base = w.pad_base; pa.pad_start = w.pad_start; pa.hdr = w.hdr;
+            pa.pad_base = r.pad_base; pa.pad_start = r.pad_start; pa.hdr = r.hdr;
             pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
             pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;

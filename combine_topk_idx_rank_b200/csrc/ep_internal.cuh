@@ -1,13 +1,10 @@
 // Internal declarations shared by the kernels and the C-ABI layer of libep.so.
 //
 // Pipeline of one dispatch (all on the caller's stream, no host sync):
-//   k_layout (one CTA per chunk of 128 or 256 tokens: validated routing,
-//   per-entry rank inside its chunk, per-chunk expert / rank histograms,
-//   is_token_in_rank) -> k_scan (expert counts, aligned expert segments,
-//   chunk row offsets, padding map, status) -> k_slots (received row of every
-//   entry, per-row metadata) -> k_pack per round (persistent: TMA bulk row
-//   copies or fused quantisation, zeroed padding rows).  Every kernel after
-//   k_layout is launched as a programmatic dependent of its predecessor.
+//   k_route (cooperative: chunk histograms and ranks | column prefixes |
+//   segment starts, received rows, per-row metadata; two grid barriers) ->
+//   k_pack per round (persistent: TMA bulk row copies or fused quantisation,
+//   zeroed padding rows), launched as a programmatic dependent.
 // Combine is one persistent kernel per round: gather + k-order fp32 FMA.
 #pragma once
 
@@ -19,26 +16,32 @@
 
 namespace ep {
 
-constexpr int kLayoutThreads = 256; // 8 warps
-constexpr int kLayoutWarps = kLayoutThreads / 32;
+constexpr int kRouteThreads = 256;  // 8 warps
+constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kMaxTopk = 16;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxRanks = 256;
 constexpr int kMaxChunkEntries = 2048;  // tokens per chunk x K
-constexpr int kMaxBatches = kMaxChunkEntries / kLayoutWarps / 32;  // 8
+constexpr int kMaxBatches = kMaxChunkEntries / kRouteWarps / 32;  // 8
 
-// Tokens per layout chunk, as a power of two: 256 (K <= 8 and R <= 64) or 128.
-inline int chunk_log2(int K, int R) { return (K <= 8 && R <= 64) ? 8 : 7; }
+// Tokens per routing chunk, as a power of two in [16, 256]: the largest with
+// C*K <= 2048 that still gives at least 128 chunks when T allows it.
+inline int chunk_log2(int T, int K) {
+    int lg = 8;
+    while ((1 << lg) * K > kMaxChunkEntries) --lg;
+    while (lg > 4 && ((T + (1 << lg) - 1) >> lg) < 128) --lg;
+    return lg;
+}
 
 // Byte offsets of the workspace regions (each 256-byte aligned).  Every
-// region is fully written before it is read within one call, so the
-// workspace never needs clearing.
+// region is written before it is read within one call (the barrier counter
+// is cleared by the call itself), so the workspace never needs clearing.
 struct WsLayout {
-    size_t hdr;          // int32[16]: [1] received rows, [2] padding rows
+    size_t hdr;          // int32[16]: [0] grid-barrier counter, [1] received rows, [2] padding rows
     size_t pad_base;     // int32[E+1] exclusive prefix sum of padding rows
     size_t pad_start;    // int32[E]   first padding row of expert e
-    size_t chunk_hist;   // int32[nchunks*E] per-chunk expert histogram
-    size_t chunk_off;    // int32[nchunks*E] row offset of (chunk, expert)
+    size_t col_total;    // int32[E+R+1] expert counts, rank counts, error flags
+    size_t chunk_hist;   // int32[nchunks*E] per-chunk expert histogram, then its prefix
     size_t chunk_rcnt;   // int32[nchunks*R] per-chunk count of tokens reaching rank r
     size_t chunk_err;    // int32[nchunks]   per-chunk status
     size_t total;
@@ -49,7 +52,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline WsLayout ws_layout(int T, int K, int E, int R) {
     WsLayout w{};
-    w.log2_chunk = chunk_log2(K, R);
+    w.log2_chunk = chunk_log2(T, K);
     const int C = 1 << w.log2_chunk;
     w.nchunks = (T + C - 1) / C;
     const size_t nc = (size_t)w.nchunks;
@@ -57,61 +60,47 @@ inline WsLayout ws_layout(int T, int K, int E, int R) {
     w.hdr = o;        o = align256(o + 16 * sizeof(int32_t));
     w.pad_base = o;   o = align256(o + sizeof(int32_t) * (E + 1));
     w.pad_start = o;  o = align256(o + sizeof(int32_t) * E);
+    w.col_total = o;  o = align256(o + sizeof(int32_t) * (E + R + 1));
     w.chunk_hist = o; o = align256(o + sizeof(int32_t) * nc * E);
-    w.chunk_off = o;  o = align256(o + sizeof(int32_t) * nc * E);
     w.chunk_rcnt = o; o = align256(o + sizeof(int32_t) * nc * R);
     w.chunk_err = o;  o = align256(o + sizeof(int32_t) * nc);
     w.total = o;
     return w;
 }
 
-struct LayoutArgs {
-    const int64_t* topk_idx;
-    int T, K, E, R, L, log2_chunk;
-    int32_t* rank_in_chunk;     // [T,K] or null
-    int32_t* chunk_hist;        // [nchunks,E]
-    uint8_t* is_token_in_rank;  // [T,R] or null
-    int32_t* topk_copy;         // [T,K] or null
-    int32_t* chunk_rcnt;        // [nchunks,R]
-    int32_t* chunk_err;         // [nchunks]
-};
-
-struct ScanArgs {
-    int E, R, A, nchunks;
-    int64_t capacity;
-    int check_capacity;
-    const int32_t* chunk_hist;   // [nchunks,E]
-    const int32_t* chunk_rcnt;   // [nchunks,R]
-    const int32_t* chunk_err;    // [nchunks]
-    int32_t* chunk_off;          // [nchunks,E] out; null = layout outputs only
-    int32_t* pad_base;           // [E+1] or null
-    int32_t* pad_start;          // [E] or null
-    int32_t* hdr;                // ws hdr: [1] rows, [2] padding rows
-    int32_t* psum;               // [E] or null
-    int32_t* num_recv;           // [E] or null
-    int32_t* num_tokens_per_expert;  // [E] or null
-    int32_t* num_tokens_per_rank;    // [R] or null
-    int32_t* cumulative;         // [E] or null
-    int32_t* err_out;            // [1]
-};
-
-struct SlotsArgs {
+struct RouteArgs {
     const int64_t* topk_idx;
     const float* topk_weights;
-    int T, K, E, L, log2_chunk;
-    int32_t* dst_slot;          // in: rank inside chunk; out: received row (-1 = none)
-    const int32_t* chunk_off;   // [nchunks,E] row offset of (chunk, expert)
+    int T, K, E, R, L, A, log2_chunk, nchunks;
+    int64_t capacity;
+    int check_capacity;
+    int assign;                 // 1: rows and metadata (dispatch); 0: layout outputs only
+    int vector_ok;              // the four [.,K] arrays are 16-byte aligned
+    int nscales;                // scales per row (0 when not quantised)
+    // per-entry / per-row outputs (dispatch)
+    int32_t* dst_slot;          // [T,K]: rank inside the chunk, then the received row
+    int32_t* topk_copy;         // [T,K] or null
     int32_t* recv_meta;
     int32_t* recv_topk_idx;
     float* recv_topk_weights;
     float* recv_scales;         // null when not quantised
-    int nscales;                // scales per row (0 when not quantised)
-    int64_t capacity;
-    const int32_t* pad_base;
-    const int32_t* pad_start;
-    const int32_t* hdr;         // [2] = padding rows
-    int max_pad;                // host bound on padding rows: E * (A - 1)
-    int vector_ok;              // the four [.,K] arrays are 16-byte aligned
+    // layout outputs (each may be null)
+    uint8_t* is_token_in_rank;  // [T,R]
+    int32_t* psum;
+    int32_t* num_recv;
+    int32_t* num_tokens_per_expert;
+    int32_t* num_tokens_per_rank;
+    int32_t* cumulative;
+    int32_t* err_out;           // [1]
+    // workspace
+    unsigned* barrier;
+    int32_t* hdr;
+    int32_t* pad_base;
+    int32_t* pad_start;
+    int32_t* col_total;
+    int32_t* chunk_hist;
+    int32_t* chunk_rcnt;
+    int32_t* chunk_err;
 };
 
 struct PackArgs {
@@ -141,9 +130,7 @@ struct CombineArgs {
 };
 
 // Launchers (return the CUDA error of the launch).
-cudaError_t launch_layout(const LayoutArgs& a, int nchunks, cudaStream_t st);
-cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
-cudaError_t launch_slots(const SlotsArgs& a, cudaStream_t st);
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

@@ -48,7 +48,7 @@ def test_host_helpers(lib):
     assert lib.ep_recv_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
     assert lib.ep_recv_capacity_bound(10, 2, 4, 1) == 20
     ws = lib.ep_workspace_bytes(32768, 8, 256, 8)
-    assert ws % 256 == 0 and ws >= 256 * 256 * 4       # chunk table of 256 chunks x 256 experts
+    assert ws % 256 == 0 and ws >= 128 * 256 * 4       # histogram of 128 chunks (256 tokens) x 256 experts
     assert lib.ep_workspace_bytes(100, 8, 256, 8) == 0  # T % R != 0 -> rejected
     assert lib.ep_workspace_bytes(64, 17, 256, 8) == 0  # K > 16
     assert lib.ep_status_string(3) == b"receive capacity too small"
