@@ -13,10 +13,17 @@
 
 #include "ep_internal.cuh"
 
+#ifndef EP_COMBINE_VPT
+#define EP_COMBINE_VPT 2   // 16-byte vectors per thread per pass (x K loads in flight)
+#endif
+#ifndef EP_COMBINE_MIN_BLOCKS
+#define EP_COMBINE_MIN_BLOCKS 1
+#endif
+
 namespace ep {
 
 template <int KMAX, int VPT>
-__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+__global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
@@ -121,7 +128,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
     const int threads = min(256, ((V + 2 * passes - 1) / (2 * passes) + 31) & ~31);
     if (a.K <= 2) return run(k_combine<2, 2>, threads, a, st);
     if (a.K <= 4) return run(k_combine<4, 2>, threads, a, st);
-    if (a.K <= 8) return run(k_combine<8, 2>, threads, a, st);
+    if (a.K <= 8) return run(k_combine<8, EP_COMBINE_VPT>, threads, a, st);
     return run(k_combine<16, 1>, threads, a, st);
 }
 

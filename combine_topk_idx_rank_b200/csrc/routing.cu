@@ -112,7 +112,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     const int C = 1 << a.log2_chunk;
     int32_t* wh = smem;                               // [8][E] per-warp running counts
     int32_t* s_idx = wh + kRouteWarps * E;            // [C*K] validated expert ids
-    int32_t* s_rcnt = s_idx + C * K;                  // [R]
+    int32_t* s_rank = s_idx + C * K;                  // [C*K] rank inside the chunk
+    float* s_w = reinterpret_cast<float*>(s_rank + C * K);   // [C*K] top-k weights
+    int32_t* s_rcnt = reinterpret_cast<int32_t*>(s_w + C * K);   // [R]
     int32_t* s_seg = s_rcnt + R;                      // [E] segment starts
     int32_t* s_al = s_seg + E;                        // [E] aligned counts, then padding prefix
     int32_t* s_pad = s_al + E;                        // [E+1] padding prefix
@@ -127,6 +129,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     const unsigned lt = lanemask_lt();
     const int per_warp = ((C * K / kRouteWarps) + 31) & ~31;   // entries per warp, a multiple of 32
     const int nb = per_warp / 32;
+    // with one chunk per CTA its ids, weights and ranks stay in shared memory
+    // from phase 1 to phase 3; otherwise phase 3 reloads them
+    const bool resident = a.nchunks <= G;
 
     // ---------------------------------------------------------------- phase 1
     for (int c = blockIdx.x; c < a.nchunks; c += G) {
@@ -138,6 +143,15 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         for (int i = tid; i < R; i += kRouteThreads) s_rcnt[i] = 0;
         for (int i = tid; i < nt * R; i += kRouteThreads) s_inr[i] = 0;
         if (tid == 0) *s_err = 0;
+        // this warp's entries (and, for dispatch, the chunk's weights), all loads issued up front
+        int64_t ld[kMaxBatches];
+#pragma unroll
+        for (int b = 0; b < kMaxBatches; ++b) {
+            const int i = warp * per_warp + b * 32 + lane;
+            ld[b] = (b < nb && i < ne) ? a.topk_idx[e0 + i] : -1;
+        }
+        if (a.assign)
+            for (int i = tid; i < ne; i += kRouteThreads) s_w[i] = a.topk_weights[e0 + i];
         __syncthreads();
         int my_e[kMaxBatches], my_r[kMaxBatches];
 #pragma unroll
@@ -148,7 +162,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 const int i = warp * per_warp + b * 32 + lane;
                 int e = -1;
                 if (i < ne) {
-                    const int64_t v = a.topk_idx[e0 + i];
+                    const int64_t v = ld[b];
                     if (v < -1 || v >= E) *s_err = EP_ERR_BAD_EXPERT_ID;
                     else e = (int)v;
                     s_idx[i] = e;
@@ -181,7 +195,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 const int i = warp * per_warp + b * 32 + lane;
                 if (i < ne) {
                     const int e = my_e[b];
-                    if (a.dst_slot) a.dst_slot[e0 + i] = e >= 0 ? wh[warp * E + e] + my_r[b] : -1;
+                    const int rank = e >= 0 ? wh[warp * E + e] + my_r[b] : -1;
+                    s_rank[i] = rank;
+                    if (a.dst_slot && !resident) a.dst_slot[e0 + i] = rank;
                     if (a.topk_copy) a.topk_copy[e0 + i] = e;
                 }
             }
@@ -286,42 +302,37 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     if (!a.assign) return;
 
     // received row of every entry, and the per-row metadata
+    int32_t* s_pre = s_al;   // [E] the chunk's column prefixes (padding counts live in s_pad now)
     for (int c = blockIdx.x; c < a.nchunks; c += G) {
         const int t0 = c * C;
         const int ne = min(C, a.T - t0) * K;
         const int64_t e0 = (int64_t)t0 * K;
-        const int32_t* pre = a.chunk_hist + (size_t)c * E;
+        __syncthreads();
+        for (int e = tid; e < E; e += kRouteThreads) s_pre[e] = __ldcg(a.chunk_hist + (size_t)c * E + e);
+        if (!resident) {
+            for (int i = tid; i < ne; i += kRouteThreads) {
+                const int64_t v = a.topk_idx[e0 + i];
+                s_idx[i] = (v >= 0 && v < E) ? (int)v : -1;
+                s_rank[i] = a.dst_slot[e0 + i];
+                s_w[i] = a.topk_weights[e0 + i];
+            }
+        }
+        __syncthreads();
         for (int i = tid; i < ne; i += kRouteThreads) {
-            const int64_t gi = e0 + i;
-            const int t = t0 + i / K, k = i - (i / K) * K;
-            const int64_t v = a.topk_idx[gi];
-            const int e = (v >= 0 && v < E) ? (int)v : -1;
+            const int tl = i / K, k = i - tl * K;
+            const int e = s_idx[i];
             int slot = -1;
             if (e >= 0) {
-                const int rank = a.dst_slot[gi];
-                const int64_t row = (int64_t)s_seg[e] + __ldcg(pre + e) + rank;
-                slot = (rank >= 0 && row < a.capacity) ? (int)row : -1;
+                const int64_t row = (int64_t)s_seg[e] + s_pre[e] + s_rank[i];
+                slot = row < a.capacity ? (int)row : -1;
             }
-            a.dst_slot[gi] = slot;
+            a.dst_slot[e0 + i] = slot;
             if (slot < 0) continue;
-            reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t, k);
+            reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t0 + tl, k);
             const int rdst = e / L;
-            const int64_t* row_ids = a.topk_idx + (int64_t)t * K;
-            const float* row_w = a.topk_weights + (int64_t)t * K;
+            const int* ids = s_idx + tl * K;
+            const float* ws = s_w + tl * K;
             if constexpr (KT > 0) {
-                int ids[KT];
-                float ws[KT];
-#pragma unroll
-                for (int j = 0; j < KT; j += 2) {
-                    const longlong2 p = __ldg(reinterpret_cast<const longlong2*>(row_ids) + j / 2);
-                    ids[j] = (p.x >= 0 && p.x < E) ? (int)p.x : -1;
-                    ids[j + 1] = (p.y >= 0 && p.y < E) ? (int)p.y : -1;
-                }
-#pragma unroll
-                for (int j = 0; j < KT; j += 4) {
-                    const float4 q = __ldg(reinterpret_cast<const float4*>(row_w) + j / 4);
-                    ws[j] = q.x; ws[j + 1] = q.y; ws[j + 2] = q.z; ws[j + 3] = q.w;
-                }
                 int4* ri = reinterpret_cast<int4*>(a.recv_topk_idx + (int64_t)slot * KT);
                 float4* rw = reinterpret_cast<float4*>(a.recv_topk_weights + (int64_t)slot * KT);
 #pragma unroll
@@ -342,10 +353,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 int32_t* ri = a.recv_topk_idx + (int64_t)slot * K;
                 float* rw = a.recv_topk_weights + (int64_t)slot * K;
                 for (int j = 0; j < K; ++j) {
-                    const int64_t ej = __ldg(row_ids + j);
-                    const bool here = ej >= 0 && ej < E && (int)ej / L == rdst;
-                    ri[j] = here ? (int)ej - rdst * L : -1;
-                    rw[j] = here ? __ldg(row_w + j) : 0.0f;
+                    const int ej = ids[j];
+                    const bool here = ej >= 0 && ej / L == rdst;
+                    ri[j] = here ? ej - rdst * L : -1;
+                    rw[j] = here ? ws[j] : 0.0f;
                 }
             }
         }
@@ -370,7 +381,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
 
 size_t route_smem_bytes(int E, int K, int R, int log2_chunk) {
     const int C = 1 << log2_chunk;
-    return sizeof(int32_t) * ((size_t)kRouteWarps * E + (size_t)C * K + R + 3 * (size_t)E + 1 + 40) +
+    return sizeof(int32_t) * ((size_t)kRouteWarps * E + 3 * (size_t)C * K + R + 3 * (size_t)E + 1 + 40) +
            (size_t)C * R;
 }
 
