@@ -17,7 +17,7 @@
 #define EP_COMBINE_VPT 2   // 16-byte vectors per thread per pass (x K loads in flight)
 #endif
 #ifndef EP_COMBINE_MIN_BLOCKS
-#define EP_COMBINE_MIN_BLOCKS 1
+#define EP_COMBINE_MIN_BLOCKS 3   // caps registers at 80: 3 CTAs of 224 threads per SM
 #endif
 
 namespace ep {

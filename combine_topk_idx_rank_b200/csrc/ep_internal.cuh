@@ -26,10 +26,13 @@ constexpr int kMaxBatches = kMaxChunkEntries / kRouteWarps / 32;  // 8
 
 // Tokens per routing chunk, as a power of two in [16, 256]: the largest with
 // C*K <= 2048 that still gives at least 128 chunks when T allows it.
+#ifndef EP_ROUTE_MIN_CHUNKS
+#define EP_ROUTE_MIN_CHUNKS 128
+#endif
 inline int chunk_log2(int T, int K) {
     int lg = 8;
     while ((1 << lg) * K > kMaxChunkEntries) --lg;
-    while (lg > 4 && ((T + (1 << lg) - 1) >> lg) < 128) --lg;
+    while (lg > 4 && ((T + (1 << lg) - 1) >> lg) < EP_ROUTE_MIN_CHUNKS) --lg;
     return lg;
 }
 
