@@ -32,7 +32,7 @@ EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, E
 _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
-            "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string")
+            "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc")
 
 
 class EPError(RuntimeError):

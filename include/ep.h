@@ -159,6 +159,27 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
                         uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Dispatch for callers that cannot allocate device memory.  The pages have no
+ * counterpart: it is ep_dispatch with the same arguments and results, minus
+ * the workspace, for code that may not call cudaMalloc (a region that must not
+ * allocate, a plugin that only receives its input and output pointers, a
+ * runtime without an allocator).  The routing scratch lives instead in one
+ * static device array of 2 MiB per GPU, held until the process exits; sizes
+ * whose scratch (ep_workspace_bytes) exceeds 2 MiB return EP_ERR_INVALID_ARG
+ * with a message on stderr, before anything runs.  The first call on a device
+ * looks up the array's address (make it before any stream capture).  All
+ * calls on a device share the array: calls whose kernels overlap on the GPU
+ * race, so serialise them on one stream.  Allocates nothing.
+ */
+ep_status_t ep_dispatch_noalloc(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                                const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                                const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                                int32_t* recv_topk_idx, float* recv_topk_weights,
+                                int64_t recv_capacity, ep_handle_t* handle,
+                                int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                                uint8_t* is_token_in_rank, void* stream);
+
+/*
  * Combine (combine, comparative analysis section 9.2): for every token t
  *   out[t] = bf16_rne( sum over k = 0..K-1 with dst_buffer_slot_idx[t,k] >= 0
  *                      of topk_weights[t,k] * y[dst_buffer_slot_idx[t,k]] ),
