@@ -26,6 +26,12 @@
 #ifndef EP_PACK_STAGES
 #define EP_PACK_STAGES 4
 #endif
+#ifndef EP_PACK_LOAD_HINT
+#define EP_PACK_LOAD_HINT 0    // 1: bulk loads of x rows carry an L2 evict-first policy
+#endif
+#ifndef EP_PACK_STORE_HINT
+#define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
+#endif
 
 namespace ep {
 
@@ -66,17 +72,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
+#if EP_PACK_LOAD_HINT || EP_PACK_STORE_HINT
+// L2 policy that marks lines for early eviction (rows are read or written once)
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+#endif
 __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+#if EP_PACK_LOAD_HINT
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(l2_evict_first())
+        : "memory");
+#else
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             smem_u32(sdst)),
         "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+#endif
 }
 __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+#if EP_PACK_STORE_HINT
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes), "l"(l2_evict_first())
+                 : "memory");
+#else
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
                  "r"(bytes)
                  : "memory");
+#endif
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
