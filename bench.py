@@ -165,6 +165,58 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sel)}
 
 
+# ------------------------------------------------------- multi-rank plumbing
+
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend: str, local: int, timeout_s: float = 120.0):
+    """Joins the process group when there is more than one rank.  Each rank
+    runs an independent problem, so the group carries only barriers and the
+    max-reduction of timings, never data."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        kw = {}
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return world, rank
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Every rank draws its own problem."""
+    return seed + rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the tokens of all ranks' problems over the
+    slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args):
@@ -173,19 +225,13 @@ def run_ours(args):
 
     from combine_topk_idx_rank_b200 import ep
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    world, rank = init_dist("nccl", local)
     dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
 
     cfg = CONFIGS[args.workload]
-    wl = make_workload(cfg, seed=args.seed + rank)
+    wl = make_workload(cfg, seed=rank_seed(args.seed, rank))
     T, H, K, E, R = cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks
     x = torch.from_numpy(wl.x.view(np.int16)).view(torch.bfloat16).to(dev)
     ti = torch.from_numpy(wl.topk_idx).to(dev)
@@ -227,8 +273,7 @@ def run_ours(args):
     bufs.handle.check()
     counts = bufs.handle.num_recv_tokens_per_expert.cpu().numpy()
 
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -237,18 +282,14 @@ def run_ours(args):
         step(i)
     stop.record()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     t_wall1 = time.time()
     sampler.stop()
     elapsed_ms = start.elapsed_time(stop)
     pack_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)) / args.steps
     combine_ms = sum(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)) / args.steps
 
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # ------------------------------------------------------------ end to end
     e2e_steps = max(3, min(args.steps, 20))
@@ -271,8 +312,7 @@ def run_ours(args):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
@@ -280,17 +320,14 @@ def run_ours(args):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = hx.numel() * 2 + hti.numel() * 8 + htw.numel() * 4
     d2h = hout.numel() * 2
 
     ab = algorithmic_bytes(cfg, counts, T)
     ms_per_step = elapsed_ms / args.steps
     step_bytes = ab["layout"] + ab["pack"] + ab["combine"]
-    value = world * T / (ms_per_step / 1e3)
+    value = job_tokens_per_s(world, T, ms_per_step)
     gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
     pack_gbs = ab["pack"] / (pack_ms * 1e-3) / 1e9
@@ -322,7 +359,7 @@ def run_ours(args):
                      "peak_kind": peak_kind, "frac": round(dom_gbs / peak, 4),
                      "algorithmic_bytes_per_launch": int(dom_bytes), "launch_ms": round(dom_ms, 5),
                      "traffic": traffic_for(dom, args.workload)},
-        "e2e": {"value": round(world * T * e2e_steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
+        "e2e": {"value": round(job_tokens_per_s(world, T, e2e_ms / e2e_steps), 1), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms / e2e_steps, 4)},
         "gpu_launches": launches_per_step * args.steps,
@@ -332,8 +369,8 @@ def run_ours(args):
         result["cpu_baseline"] = cpu_baseline(cfg, wl, budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(result), flush=True)
+    barrier(world)
     if world > 1:
-        dist.barrier()
         dist.destroy_process_group()
 
 
@@ -380,9 +417,8 @@ def cpu_baseline(cfg, wl, budget_s=15.0, quick=False):
 
 
 def run_reference(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    world, rank, _ = dist_env()
+    if rank != 0:       # under torchrun only rank 0 times the oracle
         return
     cfg = CONFIGS[args.workload]
     wl = make_workload(cfg, seed=args.seed)
