@@ -165,6 +165,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sel)}
 
 
+def workload_config(args):
+    """The named workload, optionally with a different token count (--tokens)."""
+    cfg = CONFIGS[args.workload]
+    if getattr(args, "tokens", 0):
+        if args.tokens % (cfg.num_ranks * cfg.num_rounds):
+            raise SystemExit(f"--tokens must be a multiple of ranks x rounds = {cfg.num_ranks * cfg.num_rounds}")
+        cfg = cfg.scaled(num_tokens=args.tokens)
+    return cfg
+
+
 # ------------------------------------------------------- multi-rank plumbing
 
 def dist_env():
@@ -230,7 +240,7 @@ def run_ours(args):
     world, rank = init_dist("nccl", local)
     dev = torch.device("cuda", local)
 
-    cfg = CONFIGS[args.workload]
+    cfg = workload_config(args)
     wl = make_workload(cfg, seed=rank_seed(args.seed, rank))
     T, H, K, E, R = cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks
     x = torch.from_numpy(wl.x.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -251,11 +261,20 @@ def run_ours(args):
             e.record()
     torch.cuda.synchronize()
 
-    def step(i=None):
-        evs = None if i is None else (ev[i][0], ev[i][1])
+    if args.mode == "cached":       # routing computed once; every step re-packs with the handle
         ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
                        quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
-                       do_cpu_sync=False, buffers=bufs, events=evs)
+                       do_cpu_sync=False, buffers=bufs)
+
+    def step(i=None):
+        evs = None if i is None else (ev[i][0], ev[i][1])
+        if args.mode == "cached":
+            ep.ep_dispatch(x, quant=q, quant_size=cfg.quant_size, round_scale=cfg.round_scale,
+                           num_rounds=cfg.num_rounds, buffers=bufs, events=evs, handle=bufs.handle)
+        else:
+            ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
+                           quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
+                           do_cpu_sync=False, buffers=bufs, events=evs)
         if i is not None:
             ev[i][2].record()
         ep.ep_combine(y, bufs.handle, tw, out=out)
@@ -325,6 +344,9 @@ def run_ours(args):
     d2h = hout.numel() * 2
 
     ab = algorithmic_bytes(cfg, counts, T)
+    if args.mode == "cached":
+        ab["layout"] = 0
+        ab["pack"] -= T * cfg.num_topk * 8 + ab["rows_aligned"] * (2 * cfg.num_topk * 4 + 8)   # no routing / metadata
     ms_per_step = elapsed_ms / args.steps
     step_bytes = ab["layout"] + ab["pack"] + ab["combine"]
     value = job_tokens_per_s(world, T, ms_per_step)
@@ -337,14 +359,17 @@ def run_ours(args):
     else:
         dom, dom_bytes, dom_gbs, dom_ms = "k_combine", ab["combine"] / cfg.num_rounds, combine_gbs, combine_ms / cfg.num_rounds
     clocks = sampler.summary(t_wall0, t_wall1)
-    launches_per_step = 2 + 2 * cfg.num_rounds        # layout, scan, pack x rounds, combine x rounds
+    # routing (1 cooperative kernel) unless cached, pack x rounds, combine x rounds
+    launches_per_step = (0 if args.mode == "cached" else 1) + 2 * cfg.num_rounds
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q is None else f"bf16->{q}",
         "data": "synthetic (seeded numpy PCG64; no dataset, no weights)",
-        "config": {"workload": WORKLOAD_DESC[args.workload], "name": args.workload, "tokens": T, "hidden": H,
+        "config": {"workload": WORKLOAD_DESC[args.workload] + (f" (scaled to {T} tokens)" if args.tokens else "")
+                   + (" — cached dispatch (routing reused from the handle)" if args.mode == "cached" else ""),
+                   "name": args.workload, "mode": args.mode, "tokens": T, "hidden": H,
                    "num_experts": E, "num_ranks": R, "topk": K, "expert_alignment": cfg.expert_alignment,
                    "quant": cfg.quant, "num_rounds": cfg.num_rounds, "parallelism": f"{world} independent EP problems",
                    "l2": "inputs larger than L2 (x %.0f MB, recv_x/y %.0f MB each)" % (
@@ -420,7 +445,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:       # under torchrun only rank 0 times the oracle
         return
-    cfg = CONFIGS[args.workload]
+    cfg = workload_config(args)
     wl = make_workload(cfg, seed=args.seed)
     import oracle
     from combine_topk_idx_rank_b200.workloads import make_y
@@ -477,6 +502,9 @@ def main(argv=None):
     p.add_argument("--workload", default="prefill", choices=list(CONFIGS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--tokens", type=int, default=0, help="scale the workload to this many tokens")
+    p.add_argument("--mode", default="full", choices=["full", "cached"],
+                   help="cached: time dispatch re-packing with a handle (routing computed once)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the cpu_baseline sample")
     p.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the --impl reference run")
     p.add_argument("--no-cpu-baseline", action="store_true")

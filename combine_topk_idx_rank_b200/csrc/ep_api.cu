@@ -49,14 +49,58 @@ RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const
     r.log2_chunk = L.log2_chunk;
     r.nchunks = L.nchunks;
     r.barrier = reinterpret_cast<unsigned*>(at(L.hdr));
-    r.hdr = at(L.hdr);
-    r.pad_base = at(L.pad_base);
-    r.pad_start = at(L.pad_start);
     r.col_total = at(L.col_total);
     r.chunk_hist = at(L.chunk_hist);
     r.chunk_rcnt = at(L.chunk_rcnt);
     r.chunk_err = at(L.chunk_err);
     return r;
+}
+
+// The pack kernel(s) of a dispatch: one launch per round, each a
+// programmatic dependent of the previous kernel on the stream.  Rows come
+// from handle->dst_buffer_slot_idx; the padding map from the handle's psum
+// and unaligned counts.
+ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R, int quant, int quant_size,
+                               const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st) {
+    ep_status_t s;
+    if (opts->event_pack_begin) {
+        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
+        if (s) return s;
+    }
+    if (T > 0) {
+        const int rounds = opts->num_rounds;
+        const int tpr = T / R, per_round = tpr / rounds;
+        for (int j = 0; j < rounds; ++j) {
+            PackArgs pa{};
+            pa.x = static_cast<const uint16_t*>(x);
+            pa.H = H; pa.K = K; pa.E = E;
+            pa.dst_slot = h->dst_buffer_slot_idx;
+            pa.recv_x = static_cast<uint8_t*>(recv_x); pa.recv_scales = recv_scales;
+            pa.capacity = recv_capacity;
+            pa.psum = h->psum_num_recv_tokens_per_expert; pa.cnt = h->num_recv_tokens_per_expert;
+            pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
+            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
+            pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
+            pa.err = h->err;
+            s = cuda_status(launch_pack(pa, quant, st));
+            if (s) return s;
+        }
+    }
+    if (opts->event_pack_end) {
+        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_end), st));
+        if (s) return s;
+    }
+    return EP_OK;
+}
+
+// Quantisation options shared by ep_dispatch and ep_dispatch_cached.
+bool quant_ok(int quant, int quant_size, int H, const float* recv_scales) {
+    if (quant == EP_QUANT_NONE) return true;
+    if (quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8) return false;
+    const bool group = quant_size == 16 || quant_size == 32 || quant_size == 64 || quant_size == 128 ||
+                       quant_size == 256 || quant_size == 512;
+    return H % 16 == 0 && (quant_size == H || group) && H % quant_size == 0 && recv_scales != nullptr;
 }
 
 }  // namespace
@@ -120,16 +164,8 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     if (A < 1 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
     if (ep_recv_capacity_bound(T, K, E, A) >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
     if (recv_capacity < 0 || recv_capacity >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
-    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8)
-        return EP_ERR_INVALID_ARG;
-    int quant_size = 0;
-    if (quant != EP_QUANT_NONE) {
-        quant_size = opts->quant_size;
-        const bool group = quant_size == 16 || quant_size == 32 || quant_size == 64 ||
-                           quant_size == 128 || quant_size == 256 || quant_size == 512;
-        if (H % 16 != 0 || !(quant_size == H || group) || H % quant_size != 0) return EP_ERR_INVALID_ARG;
-        if (recv_scales == nullptr) return EP_ERR_INVALID_ARG;
-    }
+    const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
+    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
         h->err == nullptr)
         return EP_ERR_INVALID_ARG;
@@ -153,13 +189,11 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     r.assign = 1;
     r.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
                   aligned16(recv_topk_weights);
-    r.nscales = quant != EP_QUANT_NONE ? H / quant_size : 0;
     r.dst_slot = h->dst_buffer_slot_idx;
     r.topk_copy = h->topk_idx;
     r.recv_meta = h->recv_src_metadata;
     r.recv_topk_idx = recv_topk_idx;
     r.recv_topk_weights = recv_topk_weights;
-    r.recv_scales = quant != EP_QUANT_NONE ? recv_scales : nullptr;
     r.is_token_in_rank = is_token_in_rank;
     r.psum = h->psum_num_recv_tokens_per_expert;
     r.num_recv = h->num_recv_tokens_per_expert;
@@ -169,33 +203,28 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     r.err_out = h->err;
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-    if (opts->event_pack_begin) {
-        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
-        if (s) return s;
-    }
-    if (T > 0) {
-        const int tpr = T / R, per_round = tpr / rounds;
-        for (int j = 0; j < rounds; ++j) {
-            PackArgs pa{};
-            pa.x = static_cast<const uint16_t*>(x);
-            pa.H = H; pa.K = K; pa.E = E;
-            pa.dst_slot = h->dst_buffer_slot_idx;
-            pa.recv_x = static_cast<uint8_t*>(recv_x); pa.recv_scales = recv_scales;
-            pa.capacity = recv_capacity;
-            pa.pad_base = r.pad_base; pa.pad_start = r.pad_start; pa.hdr = r.hdr;
-            pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
-            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
-            pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
-            pa.err = h->err;
-            s = cuda_status(launch_pack(pa, quant, st));
-            if (s) return s;
-        }
-    }
-    if (opts->event_pack_end) {
-        s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_end), st));
-        if (s) return s;
-    }
-    return EP_OK;
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, recv_capacity, h,
+                              st);
+}
+
+ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dispatch_opts_t* opts,
+                               void* recv_x, float* recv_scales, void* stream) {
+    if (h == nullptr || opts == nullptr) return EP_ERR_INVALID_ARG;
+    const int T = h->num_tokens, K = h->num_topk, E = h->num_experts, R = h->num_ranks, H = h->hidden;
+    const int rounds = opts->num_rounds;
+    if (!sizes_ok(T, K, E, R)) return EP_ERR_INVALID_ARG;
+    if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
+    const int quant = opts->quant;
+    const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
+    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
+        h->err == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || h->dst_buffer_slot_idx == nullptr)) return EP_ERR_INVALID_ARG;
+    if (h->recv_capacity > 0 && recv_x == nullptr) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, h->recv_capacity, h,
+                              static_cast<cudaStream_t>(stream));
 }
 
 ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_weights, void* out,

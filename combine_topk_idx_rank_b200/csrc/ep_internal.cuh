@@ -40,9 +40,7 @@ inline int chunk_log2(int T, int K) {
 // region is written before it is read within one call (the barrier counter
 // is cleared by the call itself), so the workspace never needs clearing.
 struct WsLayout {
-    size_t hdr;          // int32[16]: [0] grid-barrier counter, [1] received rows, [2] padding rows
-    size_t pad_base;     // int32[E+1] exclusive prefix sum of padding rows
-    size_t pad_start;    // int32[E]   first padding row of expert e
+    size_t hdr;          // int32[16]: [0] grid-barrier counter
     size_t col_total;    // int32[E+R+1] expert counts, rank counts, error flags
     size_t chunk_hist;   // int32[nchunks*E] per-chunk expert histogram, then its prefix
     size_t chunk_rcnt;   // int32[nchunks*R] per-chunk count of tokens reaching rank r
@@ -61,8 +59,6 @@ inline WsLayout ws_layout(int T, int K, int E, int R) {
     const size_t nc = (size_t)w.nchunks;
     size_t o = 0;
     w.hdr = o;        o = align256(o + 16 * sizeof(int32_t));
-    w.pad_base = o;   o = align256(o + sizeof(int32_t) * (E + 1));
-    w.pad_start = o;  o = align256(o + sizeof(int32_t) * E);
     w.col_total = o;  o = align256(o + sizeof(int32_t) * (E + R + 1));
     w.chunk_hist = o; o = align256(o + sizeof(int32_t) * nc * E);
     w.chunk_rcnt = o; o = align256(o + sizeof(int32_t) * nc * R);
@@ -79,14 +75,12 @@ struct RouteArgs {
     int check_capacity;
     int assign;                 // 1: rows and metadata (dispatch); 0: layout outputs only
     int vector_ok;              // the four [.,K] arrays are 16-byte aligned
-    int nscales;                // scales per row (0 when not quantised)
     // per-entry / per-row outputs (dispatch)
     int32_t* dst_slot;          // [T,K]: rank inside the chunk, then the received row
     int32_t* topk_copy;         // [T,K] or null
     int32_t* recv_meta;
     int32_t* recv_topk_idx;
     float* recv_topk_weights;
-    float* recv_scales;         // null when not quantised
     // layout outputs (each may be null)
     uint8_t* is_token_in_rank;  // [T,R]
     int32_t* psum;
@@ -97,9 +91,6 @@ struct RouteArgs {
     int32_t* err_out;           // [1]
     // workspace
     unsigned* barrier;
-    int32_t* hdr;
-    int32_t* pad_base;
-    int32_t* pad_start;
     int32_t* col_total;
     int32_t* chunk_hist;
     int32_t* chunk_rcnt;
@@ -113,9 +104,8 @@ struct PackArgs {
     uint8_t* recv_x;
     float* recv_scales;
     int64_t capacity;
-    const int32_t* pad_base;
-    const int32_t* pad_start;
-    const int32_t* hdr;         // [2] = padding rows
+    const int32_t* psum;        // [E] inclusive prefix of the aligned counts (handle)
+    const int32_t* cnt;         // [E] unaligned counts (handle): padding map source
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
     int32_t* err;

@@ -116,14 +116,56 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Padding map from the handle: expert e's padding rows are
+// [psum[e-1] + cnt[e], psum[e]), numbered consecutively over the experts by
+// base[e] (base[E] = all padding rows).  Any blockDim that is a multiple of
+// 32; every thread returns the number of padding rows.
+__device__ int build_pad_map(const PackArgs& a, int* s_base, int* s_start, int* s_warp) {
+    const int E = a.E, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = min(tid * per, E), e1 = min(e0 + per, E);
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) sum += (a.psum[e] - (e ? a.psum[e - 1] : 0)) - a.cnt[e];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        if (lane < nwarps) s_warp[lane] = w;
+    }
+    __syncthreads();
+    int run = incl - sum + (warp > 0 ? s_warp[warp - 1] : 0);
+    for (int e = e0; e < e1; ++e) {
+        const int lo = e ? a.psum[e - 1] : 0;
+        s_base[e] = run;
+        s_start[e] = lo + a.cnt[e];
+        run += (a.psum[e] - lo) - a.cnt[e];
+    }
+    const int total = s_warp[nwarps - 1];
+    if (tid == 0) s_base[E] = total;
+    __syncthreads();
+    return total;
+}
+
 // Padding row number p (0-based over all experts) -> its row index.
-__device__ __forceinline__ int64_t pad_row(const PackArgs& a, const int* s_pad_base, int p) {
-    int lo = 0, hi = a.E;   // the last expert with pad_base <= p
+__device__ __forceinline__ int64_t pad_row(int E, const int* s_base, const int* s_start, int p) {
+    int lo = 0, hi = E;   // the last expert with base <= p
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (s_pad_base[mid] <= p) lo = mid; else hi = mid;
+        if (s_base[mid] <= p) lo = mid; else hi = mid;
     }
-    return (int64_t)a.pad_start[lo] + (p - s_pad_base[lo]);
+    return (int64_t)s_start[lo] + (p - s_base[lo]);
 }
 
 __device__ __forceinline__ float pow2_ceil_bits(float s) {
@@ -185,11 +227,6 @@ __device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot
     if (threadIdx.x < a.K) s_slot[threadIdx.x] = a.dst_slot[(int64_t)t * a.K + threadIdx.x];
 }
 
-__device__ __forceinline__ void copy_pad_base(const PackArgs& a, int* s_pad_base) {
-    if (a.do_pad)
-        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_pad_base[i] = a.pad_base[i];
-}
-
 }  // namespace
 
 // ----------------------------------------------------- bf16: TMA bulk copy
@@ -205,6 +242,8 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * chunk_bytes);
     int* sslot = reinterpret_cast<int*>(mbar + S);                 // [S][kMaxTopk]
     int* s_pad_base = sslot + S * kMaxTopk;                          // [E+1]
+    int* s_pad_start = s_pad_base + a.E + 1;                         // [E]
+    int* s_warp = s_pad_start + a.E;                                 // [32]
     const int lane = threadIdx.x;
     const int K = a.K;
     const int64_t row_bytes = (int64_t)a.H * 2;
@@ -217,7 +256,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
         fence_mbar_init();
     }
-    copy_pad_base(a, s_pad_base);
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     __syncwarp();
 
     auto unit = [&](int j, int& t, int& c) {
@@ -294,7 +333,6 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
     __syncwarp();
 
     // padding rows: bulk stores from a zeroed stage
-    const int n_pad = a.do_pad ? a.hdr[2] : 0;
     const int pad_units = n_pad * nch;
     if ((int)blockIdx.x < pad_units) {
         for (int b = lane * 16; b < chunk_bytes; b += 32 * 16)
@@ -304,7 +342,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         if (lane == 0) {
             for (int u = blockIdx.x; u < pad_units; u += gridDim.x) {
                 const int p = u / nch, c = u - p * nch;
-                const int64_t row = pad_row(a, s_pad_base, p);
+                const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, p);
                 const int64_t off = (int64_t)c * chunk_bytes;
                 const uint32_t bytes = (uint32_t)min((int64_t)chunk_bytes, row_bytes - off);
                 if (row < a.capacity) bulk_store(a.recv_x + row * row_bytes + off, stage, bytes);
@@ -323,12 +361,10 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
-    __shared__ int s_pad_base[kMaxExperts + 1];
+    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     const int tid = threadIdx.x;
     const int V = a.H / 8;   // 16-byte vectors per row
-    const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    copy_pad_base(a, s_pad_base);
-    __syncthreads();
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
@@ -355,7 +391,7 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
                 }
             }
         } else {
-            const int64_t row = pad_row(a, s_pad_base, item - a.n_tok_items);
+            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H * 2);
                 for (int v = tid; v < V; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
@@ -373,15 +409,13 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
-    __shared__ int s_pad_base[kMaxExperts + 1];
+    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     const int tid = threadIdx.x;
     const int U = a.H / 16;
     const int nscales = a.H / G;
-    const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    copy_pad_base(a, s_pad_base);
-    __syncthreads();
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
@@ -423,10 +457,11 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
                 }
             }
         } else {
-            const int64_t row = pad_row(a, s_pad_base, item - a.n_tok_items);
+            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
+                for (int j = tid; j < nscales; j += blockDim.x) a.recv_scales[(size_t)row * nscales + j] = 0.0f;
             }
         }
         __syncthreads();
@@ -442,14 +477,12 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
     grid_launch_dependents();
     __shared__ int s_slot[kMaxTopk];
     __shared__ float s_red[33];
-    __shared__ int s_pad_base[kMaxExperts + 1];
+    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarps = blockDim.x >> 5;
     const int U = a.H / 16;
-    const int n_pad = a.do_pad ? a.hdr[2] : 0;
-    copy_pad_base(a, s_pad_base);
-    __syncthreads();
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     const int n_items = a.n_tok_items + n_pad;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item < a.n_tok_items) {
@@ -505,10 +538,11 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
                 if (tid == 0) a.recv_scales[slot] = sc;
             }
         } else {
-            const int64_t row = pad_row(a, s_pad_base, item - a.n_tok_items);
+            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
+                if (tid == 0) a.recv_scales[row] = 0.0f;
             }
         }
         __syncthreads();
@@ -566,7 +600,7 @@ cudaError_t launch_bulk(const PackArgs& a, cudaStream_t st) {
     const int nch = (int)((row_bytes + kBulkChunk - 1) / kBulkChunk);
     const int chunk = (int)(((row_bytes + nch - 1) / nch + 15) / 16 * 16);
     const size_t smem = (size_t)S * chunk + S * sizeof(uint64_t) + S * kMaxTopk * sizeof(int) +
-                        (kMaxExperts + 1) * sizeof(int);
+                        (2 * (size_t)a.E + 1 + 32) * sizeof(int);
     cudaError_t e = cudaFuncSetAttribute(k_pack_bulk<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = device_sm_count() * blocks_per_sm(k_pack_bulk<S>, 32, smem);

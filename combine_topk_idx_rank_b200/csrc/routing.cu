@@ -16,7 +16,8 @@
 //   3. every CTA scans the aligned expert counts for the segment starts;
 //      row = segment start + chunk prefix + rank inside the chunk; write
 //      dst_buffer_slot_idx, recv_src_metadata, recv_topk_idx/weights and the
-//      padding rows' metadata.  CTA 0 writes the per-expert / per-rank
+//      padding rows' metadata (their bytes and scales are zeroed by the pack
+//      kernel).  CTA 0 writes the per-expert / per-rank
 //      outputs and the status word.
 // No sort, no global atomics except the barrier counter.
 #include "ep_internal.cuh"
@@ -285,15 +286,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             if (a.num_recv) a.num_recv[e] = cnt;
             if (a.num_tokens_per_expert) a.num_tokens_per_expert[e] = cnt;
             if (a.cumulative) a.cumulative[e] += cnt;
-            if (a.pad_base) a.pad_base[e] = s_pad[e];
-            if (a.pad_start) a.pad_start[e] = s_seg[e] + cnt;
         }
         for (int r = tid; r < R; r += kRouteThreads)
             if (a.num_tokens_per_rank) a.num_tokens_per_rank[r] = __ldcg(a.col_total + E + r);
         if (tid == 0) {
-            if (a.pad_base) a.pad_base[E] = pads;
-            a.hdr[1] = rows;
-            a.hdr[2] = pads;
             int status = __ldcg(a.col_total + E + R) ? EP_ERR_BAD_EXPERT_ID : 0;
             if (status == 0 && a.check_capacity && (int64_t)rows > a.capacity) status = EP_ERR_CAPACITY;
             *a.err_out = status;
@@ -361,7 +357,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             }
         }
     }
-    // padding rows: metadata (-1, -1), recv_topk_idx -1, weight 0, scale 0
+    // padding rows: metadata (-1, -1), recv_topk_idx -1, weight 0
     for (int p = blockIdx.x * kRouteThreads + tid; p < pads; p += G * kRouteThreads) {
         int lo = 0, hi = E;   // the last expert with padding prefix <= p
         while (hi - lo > 1) {
@@ -375,7 +371,6 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             a.recv_topk_idx[row * K + j] = -1;
             a.recv_topk_weights[row * K + j] = 0.0f;
         }
-        for (int j = 0; j < a.nscales; ++j) a.recv_scales[row * a.nscales + j] = 0.0f;
     }
 }
 

@@ -32,7 +32,8 @@ EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, E
 _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
-            "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc")
+            "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
+            "ep_dispatch_cached")
 
 
 class EPError(RuntimeError):
@@ -72,6 +73,8 @@ def _load(path: str = _LIB_PATH):
     L.ep_dispatch.argtypes = [p, i32, i32, p, p, i32, i32, i32, C.POINTER(_Opts), p, p, p, p, i64,
                               C.POINTER(_Handle), p, p, p, p, sz, p]
     L.ep_dispatch.restype = C.c_int
+    L.ep_dispatch_cached.argtypes = [p, C.POINTER(_Handle), C.POINTER(_Opts), p, p, p]
+    L.ep_dispatch_cached.restype = C.c_int
     L.ep_combine.argtypes = [p, C.POINTER(_Handle), p, p, p]
     L.ep_combine.restype = C.c_int
     L.ep_read_error.argtypes = [p, p, C.POINTER(C.c_int32)]
@@ -231,20 +234,56 @@ def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: 
     return ntpr, ntpe, itr
 
 
-def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                expert_alignment: int = 1, quant: Optional[str] = None, *, num_experts: int,
-                num_ranks: int, quant_size: int = 128, round_scale: bool = False,
+def _dispatch_cached(x, handle: EPHandle, quant, quant_size, round_scale, num_rounds, buffers, events):
+    h = handle
+    if tuple(x.shape) != (h.num_tokens, h.hidden):
+        raise ValueError("x must be [num_tokens, hidden] of the handle")
+    q = None if quant in (None, "none") else quant
+    if buffers is None:
+        buffers = alloc_dispatch_buffers(h.num_tokens, h.hidden, h.num_topk, h.num_experts, h.num_ranks,
+                                         h.expert_alignment, q, quant_size, num_rounds, h.recv_capacity, x.device)
+    if buffers.recv_x.shape[0] != h.recv_capacity:
+        raise ValueError("recv_x must have the handle's recv_capacity rows")
+    opts = _Opts(h.expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds, 0,
+                 None, None if events is None else events[0].cuda_event,
+                 None if events is None else events[1].cuda_event)
+    st = _lib.ep_dispatch_cached(_ptr(x), C.byref(h._c()), C.byref(opts), _ptr(buffers.recv_x),
+                                 _ptr(buffers.recv_scales), _stream(x.device))
+    _check(st, "ep_dispatch_cached")
+    recv_x, recv_scales = buffers.recv_x, buffers.recv_scales
+    if h.num_recv_rows is not None:
+        recv_x = recv_x[:h.num_recv_rows]
+        if recv_scales is not None:
+            recv_scales = recv_scales[:h.num_recv_rows]
+    return recv_x, recv_scales, None, None, h
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
+                topk_weights: Optional[torch.Tensor] = None, expert_alignment: int = 1,
+                quant: Optional[str] = None, *, num_experts: Optional[int] = None,
+                num_ranks: Optional[int] = None, quant_size: int = 128, round_scale: bool = False,
                 num_rounds: int = 1, do_cpu_sync: bool = True,
                 recv_capacity: Optional[int] = None, buffers: Optional[DispatchBuffers] = None,
                 cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
-                layout_out: Optional[tuple] = None, events: Optional[tuple] = None):
+                layout_out: Optional[tuple] = None, events: Optional[tuple] = None,
+                handle: Optional[EPHandle] = None):
     """Dispatch: returns (recv_x, recv_scales, recv_topk_idx, recv_topk_weights, handle).
 
     With ``do_cpu_sync`` the call waits for the GPU, checks the status word and
     trims the outputs to the rows received (``handle.num_recv_rows``); without
     it the outputs have ``recv_capacity`` rows and nothing waits.
+
+    Cached mode: pass ``handle=`` (from an earlier call) and no topk_idx /
+    topk_weights; x is re-packed with the cached routing, nothing waits, and
+    recv_topk_idx / recv_topk_weights come back as None.
     """
     _need_cuda(x, "x", torch.bfloat16)
+    if handle is not None:
+        if topk_idx is not None or topk_weights is not None:
+            raise ValueError("cached dispatch takes the routing from the handle")
+        return _dispatch_cached(x, handle, quant, quant_size, round_scale, num_rounds, buffers, events)
+    if topk_idx is None or topk_weights is None or num_experts is None or num_ranks is None:
+        raise ValueError("topk_idx, topk_weights, num_experts and num_ranks are required")
     _need_cuda(topk_idx, "topk_idx", torch.int64)
     _need_cuda(topk_weights, "topk_weights", torch.float32)
     T, H = x.shape

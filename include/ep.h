@@ -159,6 +159,24 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
                         uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Cached dispatch (the cached mode of dispatch, comparative analysis sections
+ * 3.2-3.3 and 8.3): re-packs new token rows x with the routing of an earlier
+ * ep_dispatch whose handle is passed, skipping the layout, the slot
+ * assignment and any host sync -- the decode-time case where the routing of
+ * consecutive steps is unchanged.  Only recv_x (and recv_scales) are written;
+ * recv_topk_idx / recv_topk_weights and the handle keep the earlier call's
+ * contents.  Padding rows are zeroed again.
+ *   x            device bf16 [T,H] with the handle's T and H
+ *   handle       filled by ep_dispatch (read only); its err word receives
+ *                device errors of this call
+ *   opts         quant, quant_size, round_scale, num_rounds and the optional
+ *                pack events are used; expert_alignment is the handle's
+ *   recv_x, recv_scales  as in ep_dispatch, handle->recv_capacity rows
+ */
+ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* handle, const ep_dispatch_opts_t* opts,
+                               void* recv_x, float* recv_scales, void* stream);
+
+/*
  * Dispatch for callers that cannot allocate device memory.  The pages have no
  * counterpart: it is ep_dispatch with the same arguments and results, minus
  * the workspace, for code that may not call cudaMalloc (a region that must not

@@ -231,3 +231,40 @@ def test_cumulative_stats_accumulate(cuda_device):
                        cumulative_local_expert_recv_stats=stats, do_cpu_sync=False)
     ref = oracle.layout(wl.topk_idx, cfg.num_experts, cfg.num_ranks)["num_tokens_per_expert"]
     assert np.array_equal(stats.cpu().numpy(), 3 * ref)
+
+
+@pytest.mark.parametrize("name", ["prefill", "decode", "qwen3", "longseq"])
+def test_cached_dispatch_repacks_new_rows(name, cuda_device):
+    """Cached dispatch (handle reuse): new x, routing from the handle; the rows
+    equal the oracle's rows of the new x at the cached slots, padding zeroed."""
+    cfg = _small(name)
+    wl = make_workload(cfg, 0)
+    (_, _, _, _, h), _, (x, ti, tw) = gpu_dispatch(cfg, wl, cuda_device)
+    rows = h.num_recv_rows
+    wl2 = make_workload(cfg, 1)           # a later step: new activations, same routing
+    x2 = torch.from_numpy(wl2.x.view(np.int16)).view(torch.bfloat16).to(cuda_device)
+    q = None if cfg.quant == "none" else cfg.quant
+    bufs = ep.alloc_dispatch_buffers(cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks,
+                                     cfg.expert_alignment, q, cfg.quant_size, cfg.num_rounds, h.recv_capacity,
+                                     cuda_device)
+    bufs.recv_x.view(torch.uint8).fill_(0x5A)              # stale contents must not survive
+    if bufs.recv_scales is not None:
+        bufs.recv_scales.fill_(7.0)
+    rx, rs, rti, rtw, h2 = ep.ep_dispatch(x2, quant=q, quant_size=cfg.quant_size, round_scale=cfg.round_scale,
+                                          num_rounds=cfg.num_rounds, buffers=bufs, handle=h)
+    torch.cuda.synchronize()
+    h.check()
+    assert rti is None and rtw is None and h2 is h and rx.shape[0] == rows
+    slots = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, cfg.expert_alignment)
+    assert slots["num_recv_rows"] == rows
+    ref_x, ref_s = oracle.dispatch_rows(wl2.x, slots["dst_buffer_slot_idx"], cfg.quant, cfg.quant_size,
+                                        cfg.round_scale, num_rows=rows)
+    assert_rows_equal(cfg, rx, rs, ref_x, ref_s)
+
+
+def test_cached_dispatch_rejects_routing_args(cuda_device):
+    cfg = CONFIGS["tiny"]
+    wl = make_workload(cfg, 0)
+    (_, _, _, _, h), _, (x, ti, tw) = gpu_dispatch(cfg, wl, cuda_device)
+    with pytest.raises(ValueError):
+        ep.ep_dispatch(x, ti, tw, handle=h)
