@@ -57,6 +57,10 @@ def lib():
         L.oracle_combine_rows.restype = C.c_int
         L.oracle_round_tokens.argtypes = [i32, i32, i32, i32, p]
         L.oracle_round_tokens.restype = i64
+        L.oracle_ll_slots.argtypes = [p, p, i32, i32, i32, i32, i32, p, p, p, p, p, p]
+        L.oracle_ll_slots.restype = C.c_int
+        L.oracle_combine_rows_q.argtypes = [p, p, i32, i32, i64, i32, i32, i32, p, p, p, p, i64, p]
+        L.oracle_combine_rows_q.restype = C.c_int
         L.oracle_f32_to_e4m3_n.argtypes = [p, i64, p]
         L.oracle_f32_to_e4m3_n.restype = None
         L.oracle_f32_to_bf16_n.argtypes = [p, i64, p]
@@ -248,4 +252,52 @@ def combine(y, dst_buffer_slot_idx, topk_weights, num_ranks: int = 1, num_rounds
     for j in range(num_rounds):
         tok = round_tokens(T, num_ranks, num_rounds, j)
         out[tok] = combine_rows(y, dst_buffer_slot_idx, topk_weights, tokens=tok)
+    return out
+
+
+# ---------------------------------------------------------- low latency
+
+def ll_slots(topk_idx, topk_weights, num_experts: int, num_ranks: int, max_tokens_per_rank: int):
+    """Low-latency fixed-capacity layout: rows e*R*M + r*M + p (see ep_oracle.c)."""
+    ti = _c(topk_idx, np.int64)
+    tw = _c(topk_weights, np.float32)
+    T, K = ti.shape
+    E, R, M = num_experts, num_ranks, max_tokens_per_rank
+    rows = E * R * M
+    dst = np.zeros((T, K), np.int32)
+    cnt = np.zeros(E, np.int32)
+    rng = np.zeros((E, R), np.int64)
+    meta = np.full((rows, 2), -7, np.int32)          # untouched rows keep this marker
+    rti = np.full((rows, K), -7, np.int32)
+    rtw = np.full((rows, K), -7.0, np.float32)
+    st = lib().oracle_ll_slots(_ptr(ti), _ptr(tw), T, K, E, R, M, _ptr(dst), _ptr(cnt), _ptr(rng),
+                               _ptr(meta), _ptr(rti), _ptr(rtw))
+    if st:
+        raise OracleError(st, "ll_slots")
+    return {"dst_buffer_slot_idx": dst, "recv_count": cnt, "layout_range": rng, "recv_src_metadata": meta,
+            "recv_topk_idx": rti, "recv_topk_weights": rtw}
+
+
+def combine_rows_q(y, y_scales, quant: str, quant_size: int, dst_buffer_slot_idx, topk_weights,
+                   shared=None, tokens=None):
+    """Combine of quantised (or bf16) expert outputs, optionally starting from a shared-expert row."""
+    dst = _c(dst_buffer_slot_idx, np.int32)
+    tw = _c(topk_weights, np.float32)
+    T, K = dst.shape
+    if quant == "none":
+        ys = _c(y, np.uint16)
+        sc = None
+    else:
+        ys = _c(y, np.uint8)
+        sc = _c(y_scales, np.float32)
+    H = ys.shape[1]
+    sh = None if shared is None else _c(shared, np.uint16)
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tok = _c(tokens, np.int32)
+    out = np.zeros((tok.shape[0], H), np.uint16)
+    st = lib().oracle_combine_rows_q(_ptr(ys), _ptr(sc), QUANT[quant], quant_size, ys.shape[0], H, T, K,
+                                     _ptr(dst), _ptr(tw), _ptr(sh), _ptr(tok), tok.shape[0], _ptr(out))
+    if st:
+        raise OracleError(st, "combine_rows_q")
     return out

@@ -370,3 +370,88 @@ void oracle_f32_to_bf16_n(const float* x, int64_t n, uint16_t* out) {
 void oracle_e4m3_to_f64_n(const uint8_t* c, int64_t n, double* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_to_f64(c[i]);
 }
+
+/* -------------------------------------------- low-latency (fixed capacity) */
+
+/* The low-latency receive layout of the decode path (comparative analysis,
+ * section 6.3: a buffer of [num_local_experts, num_ranks *
+ * num_max_dispatch_tokens_per_rank, hidden] per rank; on one GPU the ranks'
+ * buffers stack to [E, R*M, H]).  The entry (t,k) routed to expert e from
+ * source rank r = t / (T/R) goes to row e*R*M + r*M + p, where p counts the
+ * earlier entries (t', k') of the same source rank and expert in (t, k) order.
+ * recv_count[e] = entries of expert e; layout_range[e*R + r] = (r*M << 32) |
+ * (entries of expert e from rank r).  Rows not used keep their content.
+ * Returns OR_CAPACITY if some (expert, source rank) has more than M entries. */
+int oracle_ll_slots(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R, int M,
+                    int32_t* dst_buffer_slot_idx, int32_t* recv_count, int64_t* layout_range,
+                    int32_t* recv_src_metadata, int32_t* recv_topk_idx, float* recv_topk_weights) {
+    if (T < 0 || K < 1 || E < 1 || R < 1 || E % R != 0 || T % R != 0 || M < 1) return OR_INVALID_ARG;
+    int st = check_ids(topk_idx, T, K, E);
+    if (st) return st;
+    int L = E / R, tpr = T / R;
+    for (int64_t i = 0; i < (int64_t)T * K; ++i) dst_buffer_slot_idx[i] = -1;
+    for (int e = 0; e < E; ++e) recv_count[e] = 0;
+    for (int e = 0; e < E; ++e) {
+        int r_dst = e / L;
+        for (int r = 0; r < R; ++r) {
+            int64_t p = 0;
+            for (int t = r * tpr; t < (r + 1) * tpr; ++t)
+                for (int k = 0; k < K; ++k) {
+                    if (topk_idx[(int64_t)t * K + k] != e) continue;
+                    if (p >= M) return OR_CAPACITY;
+                    int64_t row = ((int64_t)e * R + r) * M + p;
+                    dst_buffer_slot_idx[(int64_t)t * K + k] = (int32_t)row;
+                    recv_src_metadata[2 * row] = t;
+                    recv_src_metadata[2 * row + 1] = k;
+                    for (int j = 0; j < K; ++j) {
+                        int64_t ej = topk_idx[(int64_t)t * K + j];
+                        int here = ej >= 0 && ej / L == r_dst;
+                        recv_topk_idx[row * K + j] = here ? (int32_t)(ej - (int64_t)r_dst * L) : -1;
+                        recv_topk_weights[row * K + j] = here ? topk_weights[(int64_t)t * K + j] : 0.0f;
+                    }
+                    p += 1;
+                }
+            layout_range[(int64_t)e * R + r] = ((int64_t)r * M << 32) | p;
+            recv_count[e] += (int32_t)p;
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------ combine of quantised outputs */
+
+/* As oracle_combine_rows, for expert outputs given as FP8 e4m3 / int8 codes
+ * with one fp32 scale per quant_size channels (the combine-side quantisation
+ * of guide v2.1): each value is decode(code) * scale (fp32 product) before the
+ * fma chain.  quant OR_QUANT_NONE reads bf16 y.  If `shared` is given (bf16
+ * [T,H], a shared expert's output), the accumulator starts from shared[t]
+ * instead of +0. */
+int oracle_combine_rows_q(const void* y, const float* y_scales, int quant, int quant_size, int64_t y_rows,
+                          int H, int T, int K, const int32_t* dst_buffer_slot_idx, const float* topk_weights,
+                          const uint16_t* shared, const int32_t* tokens, int64_t n_tokens, uint16_t* out) {
+    if (quant != OR_QUANT_NONE && (quant_size < 1 || H % quant_size != 0)) return OR_INVALID_ARG;
+    int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int t = tokens[i];
+        if (t < 0 || t >= T) return OR_INVALID_ARG;
+        for (int h = 0; h < H; ++h) {
+            float acc = shared ? oracle_bf16_to_f32(shared[(int64_t)t * H + h]) : 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+                if (row < 0) continue;
+                if (row >= y_rows) return OR_CAPACITY;
+                float v;
+                if (quant == OR_QUANT_NONE) {
+                    v = oracle_bf16_to_f32(((const uint16_t*)y)[row * H + h]);
+                } else {
+                    uint8_t c = ((const uint8_t*)y)[row * H + h];
+                    float d = quant == OR_QUANT_FP8 ? (float)oracle_e4m3_to_f64(c) : (float)(int8_t)c;
+                    v = d * y_scales[row * ns + h / quant_size];
+                }
+                acc = fmaf(topk_weights[(int64_t)t * K + k], v, acc);
+            }
+            out[i * H + h] = oracle_f32_to_bf16(acc);
+        }
+    }
+    return OR_OK;
+}
