@@ -10,6 +10,8 @@
 // rows for its vectors before the first FMA, so each thread keeps K x VPT
 // 16-byte loads in flight.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "ep_internal.cuh"
 
@@ -22,7 +24,33 @@
 
 namespace ep {
 
-template <int KMAX, int VPT>
+// YQ: 0 = bf16 expert outputs; 1 = FP8 e4m3 codes, 2 = int8 codes, each value
+// decode(code) * scale (fp32 product) with one fp32 scale per quant_size
+// channels.  With a shared-expert row the accumulator starts from it.
+template <int YQ>
+__device__ __forceinline__ void dequant8(uint2 c, float s, float (&v)[8]) {
+    const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if constexpr (YQ == 1) {
+            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[h] & 0xffffu), __NV_E4M3);
+            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[h] >> 16), __NV_E4M3);
+            v[4 * h + 0] = __half2float(__ushort_as_half(lo.x));
+            v[4 * h + 1] = __half2float(__ushort_as_half(lo.y));
+            v[4 * h + 2] = __half2float(__ushort_as_half(hi.x));
+            v[4 * h + 3] = __half2float(__ushort_as_half(hi.y));
+        } else {
+            v[4 * h + 0] = (float)(int8_t)(w[h] & 0xff);
+            v[4 * h + 1] = (float)(int8_t)((w[h] >> 8) & 0xff);
+            v[4 * h + 2] = (float)(int8_t)((w[h] >> 16) & 0xff);
+            v[4 * h + 3] = (float)(int8_t)(w[h] >> 24);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], s);
+}
+
+template <int KMAX, int VPT, int YQ>
 __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
@@ -30,7 +58,8 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
     __shared__ float s_w[kMaxTopk];
     __shared__ int s_n;
     const int tid = threadIdx.x, lane = tid & 31;
-    const int V = a.H / 8;
+    const int V = a.H / 8;                              // slots of 8 channels per row
+    const int nscales = YQ ? a.H / a.quant_size : 0;
     for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
         const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
         if (tid < 32) {
@@ -56,15 +85,26 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
         const int n = s_n;
         uint16_t* orow = a.out + (size_t)t * a.H;
         for (int v0 = 0; v0 < V; v0 += VPT * blockDim.x) {
+            // every load of the pass is issued before the first FMA
             uint4 r[VPT][KMAX];
+            uint2 q[VPT][KMAX];
+            float sc[VPT][KMAX];
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
                 if (j < n) {
-                    const uint4* yr = reinterpret_cast<const uint4*>(a.y + (size_t)s_slot[j] * a.H);
 #pragma unroll
                     for (int u = 0; u < VPT; ++u) {
                         const int v = v0 + u * blockDim.x + tid;
-                        if (v < V) r[u][j] = ld_nc_v4(yr + v);
+                        if (v < V) {
+                            if constexpr (YQ == 0) {
+                                const uint16_t* yr = reinterpret_cast<const uint16_t*>(a.y) + (size_t)s_slot[j] * a.H;
+                                r[u][j] = ld_nc_v4(reinterpret_cast<const uint4*>(yr) + v);
+                            } else {
+                                const uint8_t* yr = reinterpret_cast<const uint8_t*>(a.y) + (size_t)s_slot[j] * a.H;
+                                q[u][j] = __ldg(reinterpret_cast<const uint2*>(yr) + v);
+                                sc[u][j] = __ldg(a.y_scales + (size_t)s_slot[j] * nscales + (v * 8) / a.quant_size);
+                            }
+                        }
                     }
                 }
             }
@@ -72,21 +112,28 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
             for (int u = 0; u < VPT; ++u) {
                 const int v = v0 + u * blockDim.x + tid;
                 float acc[8];
+                if (a.shared != nullptr && v < V) {
+                    const uint4 b = ld_nc_v4(reinterpret_cast<const uint4*>(a.shared + (size_t)t * a.H) + v);
+                    acc[0] = bf16lo(b.x); acc[1] = bf16hi(b.x); acc[2] = bf16lo(b.y); acc[3] = bf16hi(b.y);
+                    acc[4] = bf16lo(b.z); acc[5] = bf16hi(b.z); acc[6] = bf16lo(b.w); acc[7] = bf16hi(b.w);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+                    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+                }
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (j < n) {
                         const float w = s_w[j];
-                        const uint4 q = r[u][j];
-                        acc[0] = __fmaf_rn(w, bf16lo(q.x), acc[0]);
-                        acc[1] = __fmaf_rn(w, bf16hi(q.x), acc[1]);
-                        acc[2] = __fmaf_rn(w, bf16lo(q.y), acc[2]);
-                        acc[3] = __fmaf_rn(w, bf16hi(q.y), acc[3]);
-                        acc[4] = __fmaf_rn(w, bf16lo(q.z), acc[4]);
-                        acc[5] = __fmaf_rn(w, bf16hi(q.z), acc[5]);
-                        acc[6] = __fmaf_rn(w, bf16lo(q.w), acc[6]);
-                        acc[7] = __fmaf_rn(w, bf16hi(q.w), acc[7]);
+                        float y[8];
+                        if constexpr (YQ == 0) {
+                            const uint4 b = r[u][j];
+                            y[0] = bf16lo(b.x); y[1] = bf16hi(b.x); y[2] = bf16lo(b.y); y[3] = bf16hi(b.y);
+                            y[4] = bf16lo(b.z); y[5] = bf16hi(b.z); y[6] = bf16lo(b.w); y[7] = bf16hi(b.w);
+                        } else {
+                            dequant8<YQ>(q[u][j], sc[u][j], y);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, y[i], acc[i]);
                     }
                 }
                 if (v < V) {
@@ -126,10 +173,18 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
     // 2 vectors per thread per pass; split the row into equal passes
     const int passes = (V + 2 * 256 - 1) / (2 * 256);
     const int threads = min(256, ((V + 2 * passes - 1) / (2 * passes) + 31) & ~31);
-    if (a.K <= 2) return run(k_combine<2, 2>, threads, a, st);
-    if (a.K <= 4) return run(k_combine<4, 2>, threads, a, st);
-    if (a.K <= 8) return run(k_combine<8, EP_COMBINE_VPT>, threads, a, st);
-    return run(k_combine<16, 1>, threads, a, st);
+    if (a.y_quant == EP_QUANT_FP8_E4M3) {
+        if (a.K <= 8) return run(k_combine<8, 2, 1>, threads, a, st);
+        return run(k_combine<16, 1, 1>, threads, a, st);
+    }
+    if (a.y_quant == EP_QUANT_INT8) {
+        if (a.K <= 8) return run(k_combine<8, 2, 2>, threads, a, st);
+        return run(k_combine<16, 1, 2>, threads, a, st);
+    }
+    if (a.K <= 2) return run(k_combine<2, 2, 0>, threads, a, st);
+    if (a.K <= 4) return run(k_combine<4, 2, 0>, threads, a, st);
+    if (a.K <= 8) return run(k_combine<8, EP_COMBINE_VPT, 0>, threads, a, st);
+    return run(k_combine<16, 1, 0>, threads, a, st);
 }
 
 }  // namespace ep

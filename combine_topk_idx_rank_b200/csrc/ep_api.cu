@@ -48,6 +48,8 @@ RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const
     r.T = T; r.K = K; r.E = E; r.R = R; r.L = E / R; r.A = 1;
     r.log2_chunk = L.log2_chunk;
     r.nchunks = L.nchunks;
+    r.tokens_per_rank = R > 0 ? T / R : 0;
+    r.chunks_per_rank = L.chunks_per_rank;
     r.barrier = reinterpret_cast<unsigned*>(at(L.hdr));
     r.col_total = at(L.col_total);
     r.chunk_hist = at(L.chunk_hist);
@@ -80,7 +82,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.capacity = recv_capacity;
             pa.psum = h->psum_num_recv_tokens_per_expert; pa.cnt = h->num_recv_tokens_per_expert;
             pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
-            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0);
+            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0) && !h->low_latency;
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.err = h->err;
             s = cuda_status(launch_pack(pa, quant, st));
@@ -181,6 +183,7 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
     h->hidden = H; h->expert_alignment = A; h->num_rounds = rounds; h->recv_capacity = recv_capacity;
+    h->low_latency = 0;
 
     RouteArgs r = route_args(ws, L, topk_idx, topk_weights, T, K, E, R);
     r.A = A;
@@ -207,6 +210,60 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
                               st);
 }
 
+ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                                    const float* topk_weights, int32_t K, int32_t E, int32_t R, int32_t M,
+                                    const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                                    int32_t* recv_topk_idx, float* recv_topk_weights, int32_t* packed_recv_count,
+                                    int64_t* packed_recv_layout_range, ep_handle_t* h, void* ws, size_t ws_bytes,
+                                    void* stream) {
+    if (!sizes_ok(T, K, E, R) || opts == nullptr || h == nullptr) return EP_ERR_INVALID_ARG;
+    if (H < 8 || H > 65536 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    const int rounds = opts->num_rounds;
+    if (opts->expert_alignment != 1 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
+    if (M < 1 || M < T / R) return EP_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)E * R * M;
+    if (rows >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
+    const int quant = opts->quant;
+    const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
+    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
+        h->err == nullptr || h->recv_src_metadata == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && h->dst_buffer_slot_idx == nullptr) return EP_ERR_INVALID_ARG;
+    if (recv_x == nullptr || recv_topk_idx == nullptr || recv_topk_weights == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || topk_idx == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, K, E, R);
+    if (ws == nullptr || ws_bytes < L.total) return EP_ERR_INVALID_ARG;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
+    h->hidden = H; h->expert_alignment = 1; h->num_rounds = rounds; h->recv_capacity = rows;
+    h->low_latency = 1;
+
+    RouteArgs r = route_args(ws, L, topk_idx, topk_weights, T, K, E, R);
+    r.capacity = rows;
+    r.check_capacity = 1;
+    r.assign = 1;
+    r.ll_M = M;
+    r.layout_range = packed_recv_layout_range;
+    r.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
+                  aligned16(recv_topk_weights);
+    r.dst_slot = h->dst_buffer_slot_idx;
+    r.topk_copy = h->topk_idx;
+    r.recv_meta = h->recv_src_metadata;
+    r.recv_topk_idx = recv_topk_idx;
+    r.recv_topk_weights = recv_topk_weights;
+    r.psum = h->psum_num_recv_tokens_per_expert;
+    r.num_recv = h->num_recv_tokens_per_expert;
+    r.num_tokens_per_expert = packed_recv_count;
+    r.cumulative = opts->cumulative_local_expert_recv_stats;
+    r.err_out = h->err;
+    ep_status_t s = cuda_status(launch_route(r, st));
+    if (s) return s;
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st);
+}
+
 ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dispatch_opts_t* opts,
                                void* recv_x, float* recv_scales, void* stream) {
     if (h == nullptr || opts == nullptr) return EP_ERR_INVALID_ARG;
@@ -227,24 +284,29 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
                               static_cast<cudaStream_t>(stream));
 }
 
-ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_weights, void* out,
-                       void* stream) {
+ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,
+                          const ep_handle_t* h, const float* topk_weights, const void* shared, void* out,
+                          void* stream) {
     if (h == nullptr) return EP_ERR_INVALID_ARG;
     const int T = h->num_tokens, K = h->num_topk, H = h->hidden, R = h->num_ranks;
     const int rounds = h->num_rounds;
     if (!sizes_ok(T, K, h->num_experts, R)) return EP_ERR_INVALID_ARG;
     if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
     if (h->err == nullptr) return EP_ERR_INVALID_ARG;
+    const int qs = y_quant == EP_QUANT_NONE ? 0 : y_quant_size;
+    if (!quant_ok(y_quant, qs, H, y_quant == EP_QUANT_NONE ? nullptr : y_scales)) return EP_ERR_INVALID_ARG;
     if (T > 0 && (out == nullptr || topk_weights == nullptr || h->dst_buffer_slot_idx == nullptr))
         return EP_ERR_INVALID_ARG;
     if (h->recv_capacity > 0 && y == nullptr) return EP_ERR_INVALID_ARG;
-    if (!aligned16(y) || !aligned16(out)) return EP_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out) || !aligned16(shared)) return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int tpr = T / R, per_round = tpr / rounds;
     for (int j = 0; j < rounds; ++j) {
         CombineArgs ca{};
-        ca.y = static_cast<const uint16_t*>(y); ca.y_rows = h->recv_capacity;
+        ca.y = y; ca.y_scales = y_scales; ca.y_quant = y_quant; ca.quant_size = qs;
+        ca.shared = static_cast<const uint16_t*>(shared);
+        ca.y_rows = h->recv_capacity;
         ca.H = H; ca.K = K; ca.T = T;
         ca.dst_slot = h->dst_buffer_slot_idx; ca.topk_weights = topk_weights;
         ca.out = static_cast<uint16_t*>(out);
@@ -254,6 +316,11 @@ ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_we
         if (s) return s;
     }
     return EP_OK;
+}
+
+ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_weights, void* out,
+                       void* stream) {
+    return ep_combine_ex(y, nullptr, EP_QUANT_NONE, 0, h, topk_weights, nullptr, out, stream);
 }
 
 ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status) {

@@ -46,7 +46,7 @@ struct WsLayout {
     size_t chunk_rcnt;   // int32[nchunks*R] per-chunk count of tokens reaching rank r
     size_t chunk_err;    // int32[nchunks]   per-chunk status
     size_t total;
-    int nchunks, log2_chunk;
+    int nchunks, log2_chunk, chunks_per_rank;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -55,7 +55,9 @@ inline WsLayout ws_layout(int T, int K, int E, int R) {
     WsLayout w{};
     w.log2_chunk = chunk_log2(T, K);
     const int C = 1 << w.log2_chunk;
-    w.nchunks = (T + C - 1) / C;
+    const int tpr = R > 0 ? T / R : 0;
+    w.chunks_per_rank = (tpr + C - 1) / C;   // chunks never straddle a source rank
+    w.nchunks = R * w.chunks_per_rank;
     const size_t nc = (size_t)w.nchunks;
     size_t o = 0;
     w.hdr = o;        o = align256(o + 16 * sizeof(int32_t));
@@ -71,6 +73,9 @@ struct RouteArgs {
     const int64_t* topk_idx;
     const float* topk_weights;
     int T, K, E, R, L, A, log2_chunk, nchunks;
+    int tokens_per_rank, chunks_per_rank;
+    int ll_M;                   // > 0: low-latency layout with this many rows per (expert, source rank)
+    int64_t* layout_range;      // [E,R] (low-latency layout) or null
     int64_t capacity;
     int check_capacity;
     int assign;                 // 1: rows and metadata (dispatch); 0: layout outputs only
@@ -112,7 +117,10 @@ struct PackArgs {
 };
 
 struct CombineArgs {
-    const uint16_t* y;
+    const void* y;              // bf16 rows, or 1-byte codes when y_quant != 0
+    const float* y_scales;      // [rows, H / quant_size] when y_quant != 0
+    int y_quant, quant_size;
+    const uint16_t* shared;     // [T,H] bf16 shared-expert rows, or null
     int64_t y_rows;
     int H, K, T;
     const int32_t* dst_slot;

@@ -135,9 +135,12 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     const bool resident = a.nchunks <= G;
 
     // ---------------------------------------------------------------- phase 1
+    // the status word of this call starts clear; every later error is first-wins
+    if (blockIdx.x == 0 && tid == 0) *a.err_out = 0;
     for (int c = blockIdx.x; c < a.nchunks; c += G) {
-        const int t0 = c * C;
-        const int nt = min(C, a.T - t0);
+        // chunks never straddle a source rank: chunk c is piece c % cpr of rank c / cpr
+        const int t0 = (c / a.chunks_per_rank) * a.tokens_per_rank + (c % a.chunks_per_rank) * C;
+        const int nt = min(C, a.tokens_per_rank - (c % a.chunks_per_rank) * C);
         const int ne = nt * K;
         const int64_t e0 = (int64_t)t0 * K;
         for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wh[i] = 0;
@@ -291,8 +294,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             if (a.num_tokens_per_rank) a.num_tokens_per_rank[r] = __ldcg(a.col_total + E + r);
         if (tid == 0) {
             int status = __ldcg(a.col_total + E + R) ? EP_ERR_BAD_EXPERT_ID : 0;
-            if (status == 0 && a.check_capacity && (int64_t)rows > a.capacity) status = EP_ERR_CAPACITY;
-            *a.err_out = status;
+            if (status == 0 && a.check_capacity && a.ll_M == 0 && (int64_t)rows > a.capacity)
+                status = EP_ERR_CAPACITY;
+            if (status) set_error(a.err_out, status);
         }
     }
     if (!a.assign) return;
@@ -300,11 +304,19 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     // received row of every entry, and the per-row metadata
     int32_t* s_pre = s_al;   // [E] the chunk's column prefixes (padding counts live in s_pad now)
     for (int c = blockIdx.x; c < a.nchunks; c += G) {
-        const int t0 = c * C;
-        const int ne = min(C, a.T - t0) * K;
+        const int r_src = c / a.chunks_per_rank;
+        const int t0 = r_src * a.tokens_per_rank + (c % a.chunks_per_rank) * C;
+        const int ne = min(C, a.tokens_per_rank - (c % a.chunks_per_rank) * C) * K;
         const int64_t e0 = (int64_t)t0 * K;
         __syncthreads();
-        for (int e = tid; e < E; e += kRouteThreads) s_pre[e] = __ldcg(a.chunk_hist + (size_t)c * E + e);
+        if (a.ll_M) {
+            // position inside (expert, source rank) = prefix from the rank's first chunk
+            const size_t c0 = (size_t)r_src * a.chunks_per_rank;
+            for (int e = tid; e < E; e += kRouteThreads)
+                s_pre[e] = __ldcg(a.chunk_hist + (size_t)c * E + e) - __ldcg(a.chunk_hist + c0 * E + e);
+        } else {
+            for (int e = tid; e < E; e += kRouteThreads) s_pre[e] = __ldcg(a.chunk_hist + (size_t)c * E + e);
+        }
         if (!resident) {
             for (int i = tid; i < ne; i += kRouteThreads) {
                 const int64_t v = a.topk_idx[e0 + i];
@@ -319,8 +331,17 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             const int e = s_idx[i];
             int slot = -1;
             if (e >= 0) {
-                const int64_t row = (int64_t)s_seg[e] + s_pre[e] + s_rank[i];
-                slot = row < a.capacity ? (int)row : -1;
+                if (a.ll_M) {
+                    const int pos = s_pre[e] + s_rank[i];
+                    if (pos < a.ll_M) {
+                        slot = (int)(((int64_t)e * R + r_src) * a.ll_M + pos);
+                    } else {
+                        set_error(a.err_out, EP_ERR_CAPACITY);
+                    }
+                } else {
+                    const int64_t row = (int64_t)s_seg[e] + s_pre[e] + s_rank[i];
+                    slot = row < a.capacity ? (int)row : -1;
+                }
             }
             a.dst_slot[e0 + i] = slot;
             if (slot < 0) continue;
@@ -356,6 +377,19 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 }
             }
         }
+    }
+    if (a.ll_M) {
+        // per (expert, source rank): (first row of the rank's block << 32) | entries
+        for (int i = blockIdx.x * kRouteThreads + tid; i < E * R; i += G * kRouteThreads) {
+            const int e = i / R, r = i - e * R;
+            const bool any = a.chunks_per_rank > 0;
+            const int lo = any ? __ldcg(a.chunk_hist + (size_t)r * a.chunks_per_rank * E + e) : 0;
+            const int hi = !any ? 0
+                           : r + 1 < R ? __ldcg(a.chunk_hist + (size_t)(r + 1) * a.chunks_per_rank * E + e)
+                                       : s_cnt[e];
+            if (a.layout_range) a.layout_range[i] = ((int64_t)r * a.ll_M << 32) | (int64_t)(hi - lo);
+        }
+        return;   // no padding rows in the fixed-capacity layout
     }
     // padding rows: metadata (-1, -1), recv_topk_idx -1, weight 0
     for (int p = blockIdx.x * kRouteThreads + tid; p < pads; p += G * kRouteThreads) {

@@ -33,7 +33,7 @@ _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
-            "ep_dispatch_cached")
+            "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex")
 
 
 class EPError(RuntimeError):
@@ -52,7 +52,7 @@ class _Opts(C.Structure):
 class _Handle(C.Structure):
     _fields_ = [("num_tokens", C.c_int32), ("num_topk", C.c_int32), ("num_experts", C.c_int32),
                 ("num_ranks", C.c_int32), ("hidden", C.c_int32), ("expert_alignment", C.c_int32),
-                ("num_rounds", C.c_int32), ("reserved", C.c_int32), ("recv_capacity", C.c_int64),
+                ("num_rounds", C.c_int32), ("low_latency", C.c_int32), ("recv_capacity", C.c_int64),
                 ("topk_idx", C.c_void_p), ("psum_num_recv_tokens_per_expert", C.c_void_p),
                 ("num_recv_tokens_per_expert", C.c_void_p), ("recv_src_metadata", C.c_void_p),
                 ("dst_buffer_slot_idx", C.c_void_p), ("err", C.c_void_p)]
@@ -75,6 +75,11 @@ def _load(path: str = _LIB_PATH):
     L.ep_dispatch.restype = C.c_int
     L.ep_dispatch_cached.argtypes = [p, C.POINTER(_Handle), C.POINTER(_Opts), p, p, p]
     L.ep_dispatch_cached.restype = C.c_int
+    L.ep_dispatch_low_latency.argtypes = [p, i32, i32, p, p, i32, i32, i32, i32, C.POINTER(_Opts), p, p, p, p,
+                                          p, p, C.POINTER(_Handle), p, sz, p]
+    L.ep_dispatch_low_latency.restype = C.c_int
+    L.ep_combine_ex.argtypes = [p, p, i32, i32, C.POINTER(_Handle), p, p, p, p]
+    L.ep_combine_ex.restype = C.c_int
     L.ep_combine.argtypes = [p, C.POINTER(_Handle), p, p, p]
     L.ep_combine.restype = C.c_int
     L.ep_read_error.argtypes = [p, p, C.POINTER(C.c_int32)]
@@ -142,12 +147,14 @@ class EPHandle:
     err: torch.Tensor                               # [1] int32
     num_recv_tokens_per_expert_list: Optional[List[int]] = None
     num_recv_rows: Optional[int] = None
+    low_latency: int = 0
 
     def _c(self) -> _Handle:
         h = _Handle()
         h.num_tokens, h.num_topk, h.num_experts = self.num_tokens, self.num_topk, self.num_experts
         h.num_ranks, h.hidden, h.expert_alignment = self.num_ranks, self.hidden, self.expert_alignment
         h.num_rounds, h.recv_capacity = self.num_rounds, self.recv_capacity
+        h.low_latency = self.low_latency
         h.topk_idx = self.topk_idx.data_ptr()
         h.psum_num_recv_tokens_per_expert = self.psum_num_recv_tokens_per_expert.data_ptr()
         h.num_recv_tokens_per_expert = self.num_recv_tokens_per_expert.data_ptr()
@@ -329,19 +336,99 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
 
 
 def ep_combine(y: torch.Tensor, handle: EPHandle, topk_weights: torch.Tensor,
-               out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Combine: out[t] = bf16(sum_k w[t,k] * y[dst_buffer_slot_idx[t,k]]), fp32 in k order."""
-    _need_cuda(y, "y", torch.bfloat16)
+               out: Optional[torch.Tensor] = None, *, y_scales: Optional[torch.Tensor] = None,
+               quant_size: int = 128, shared: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Combine: out[t] = bf16(sum_k w[t,k] * y[dst_buffer_slot_idx[t,k]]), fp32 in k order.
+
+    y may be bf16, or FP8 e4m3 / int8 codes with ``y_scales`` (one fp32 scale per
+    ``quant_size`` channels; value = code * scale).  ``shared`` (bf16 [T, H]) is
+    a shared expert's output the sum starts from.
+    """
     _need_cuda(topk_weights, "topk_weights", torch.float32)
     h = handle
+    if y.dim() == 3:                      # the low-latency layout [E, R*M, H]
+        y = y.reshape(-1, y.shape[-1])
+    if y.dtype == torch.bfloat16:
+        yq, qs = 0, 0
+    elif y.dtype in (torch.float8_e4m3fn, torch.int8):
+        if y_scales is None:
+            raise ValueError("quantised y needs y_scales")
+        _need_cuda(y_scales, "y_scales", torch.float32)
+        yq, qs = (1 if y.dtype == torch.float8_e4m3fn else 2), quant_size
+    else:
+        raise ValueError(f"unsupported y dtype {y.dtype}")
+    _need_cuda(y, "y")
     if y.shape[1] != h.hidden or y.shape[0] > h.recv_capacity:
         raise ValueError("y must be [rows <= recv_capacity, hidden] in received-row order")
     if tuple(topk_weights.shape) != (h.num_tokens, h.num_topk):
         raise ValueError("topk_weights shape does not match the handle")
+    if shared is not None:
+        _need_cuda(shared, "shared", torch.bfloat16)
+        if tuple(shared.shape) != (h.num_tokens, h.hidden):
+            raise ValueError("shared must be [num_tokens, hidden]")
     if out is None:
         out = torch.empty((h.num_tokens, h.hidden), dtype=torch.bfloat16, device=y.device)
     ch = h._c()
     ch.recv_capacity = y.shape[0]
-    st = _lib.ep_combine(_ptr(y), C.byref(ch), _ptr(topk_weights), _ptr(out), _stream(y.device))
-    _check(st, "ep_combine")
+    if yq == 0 and shared is None:
+        st = _lib.ep_combine(_ptr(y), C.byref(ch), _ptr(topk_weights), _ptr(out), _stream(y.device))
+        _check(st, "ep_combine")
+    else:
+        st = _lib.ep_combine_ex(_ptr(y), _ptr(y_scales), yq, qs, C.byref(ch), _ptr(topk_weights), _ptr(shared),
+                                _ptr(out), _stream(y.device))
+        _check(st, "ep_combine_ex")
     return out
+
+
+def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                            num_max_dispatch_tokens_per_rank: int, num_experts: int, num_ranks: int,
+                            quant: Optional[str] = None, *, quant_size: int = 128, round_scale: bool = False,
+                            workspace: Optional[torch.Tensor] = None, buffers: Optional[dict] = None,
+                            cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None):
+    """Low-latency (decode) dispatch into fixed-capacity per-expert buffers.
+
+    Returns (recv_x [E, R*M, H], recv_scales [E, R*M, H/quant_size] or None,
+    packed_recv_count [E], packed_recv_layout_range [E, R] int64, handle);
+    entry (t,k) of source rank r for expert e is row r*M + p of expert e's
+    block, p its position among rank r's entries for e.
+    """
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(topk_idx, "topk_idx", torch.int64)
+    _need_cuda(topk_weights, "topk_weights", torch.float32)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    E, R, M = num_experts, num_ranks, num_max_dispatch_tokens_per_rank
+    rows = E * R * M
+    q = None if quant in (None, "none") else quant
+    dev = x.device
+    b = buffers
+    if b is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        b = {"recv_x": torch.empty((rows, H), dtype=(torch.bfloat16 if q is None else
+                                                      torch.float8_e4m3fn if q == "fp8" else torch.int8), device=dev),
+             "recv_scales": None if q is None else torch.empty((rows, H // quant_size), dtype=torch.float32,
+                                                                device=dev),
+             "recv_topk_idx": torch.empty((rows, K), **i32),
+             "recv_topk_weights": torch.empty((rows, K), dtype=torch.float32, device=dev),
+             "count": torch.empty((E,), **i32),
+             "layout_range": torch.empty((E, R), dtype=torch.int64, device=dev),
+             "handle": EPHandle(T, K, E, R, H, 1, 1, rows, torch.empty((T, K), **i32), torch.empty((E,), **i32),
+                                torch.empty((E,), **i32), torch.empty((rows, 2), **i32),
+                                torch.empty((T, K), **i32), torch.zeros((1,), **i32), low_latency=1)}
+    h = b["handle"]
+    nbytes = workspace_bytes(T, K, E, R)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
+    opts = _Opts(1, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), 1, 0,
+                 None if cumulative_local_expert_recv_stats is None
+                 else cumulative_local_expert_recv_stats.data_ptr(), None, None)
+    ch = h._c()
+    st = _lib.ep_dispatch_low_latency(_ptr(x), T, H, _ptr(topk_idx), _ptr(topk_weights), K, E, R, M, C.byref(opts),
+                                      _ptr(b["recv_x"]), _ptr(b["recv_scales"]), _ptr(b["recv_topk_idx"]),
+                                      _ptr(b["recv_topk_weights"]), _ptr(b["count"]), _ptr(b["layout_range"]),
+                                      C.byref(ch), _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(st, "ep_dispatch_low_latency")
+    h.recv_capacity, h.low_latency, h.expert_alignment = ch.recv_capacity, 1, 1
+    rs = b["recv_scales"]
+    return (b["recv_x"].view(E, R * M, H), None if rs is None else rs.view(E, R * M, -1), b["count"],
+            b["layout_range"], h)

@@ -89,7 +89,9 @@ typedef struct {
  * to ep_combine.  ep_dispatch sets the scalar fields. */
 typedef struct {
     int32_t num_tokens, num_topk, num_experts, num_ranks, hidden, expert_alignment;
-    int32_t num_rounds, reserved;
+    int32_t num_rounds;
+    int32_t low_latency;                         /* 1: rows in the fixed-capacity layout of
+                                                    ep_dispatch_low_latency (no padding rows) */
     int64_t recv_capacity;                       /* rows of recv_x / y */
     int32_t* topk_idx;                           /* [T,K] copy of the routing as int32
                                                     (-1 = masked); may be NULL */
@@ -159,6 +161,37 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
                         uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Low-latency dispatch (the decode-mode layout: low_latency_dispatch of
+ * "DeepEP communication library guide v2.1", its fixed-capacity per-rank
+ * buffers [num_local_experts, num_ranks * num_max_dispatch_tokens_per_rank,
+ * hidden] of comparative analysis section 6.3).  On one GPU the ranks'
+ * buffers stack to recv_x [E, R*M, H] (M = num_max_dispatch_tokens_per_rank):
+ * the entry (t,k) for expert e from source rank r = t / (T/R) goes to row
+ * e*R*M + r*M + p, p its position among rank r's entries for e in (t,k) order.
+ * No global scan, no padding rows; rows past an (expert, rank) block's count
+ * are left as they were.
+ *   num_max_dispatch_tokens_per_rank  M >= T/R
+ *   recv_x, recv_scales, recv_topk_idx, recv_topk_weights  as in ep_dispatch,
+ *                        with E*R*M rows
+ *   packed_recv_count    device int32 [E]: entries received per expert (may be NULL)
+ *   packed_recv_layout_range  device int64 [E,R]: (r*M << 32) | entries from
+ *                        rank r (may be NULL)
+ *   handle               as in ep_dispatch (recv_src_metadata has E*R*M rows);
+ *                        low_latency = 1, recv_capacity = E*R*M; psum holds the
+ *                        inclusive prefix of the unaligned counts
+ * opts->expert_alignment must be 1.  More than M entries of one (expert, rank)
+ * set EP_ERR_CAPACITY (they are dropped).  ep_combine and ep_dispatch_cached
+ * accept the handle.
+ */
+ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                                    const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                                    int32_t num_max_dispatch_tokens_per_rank, const ep_dispatch_opts_t* opts,
+                                    void* recv_x, float* recv_scales, int32_t* recv_topk_idx,
+                                    float* recv_topk_weights, int32_t* packed_recv_count,
+                                    int64_t* packed_recv_layout_range, ep_handle_t* handle, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/*
  * Cached dispatch (the cached mode of dispatch, comparative analysis sections
  * 3.2-3.3 and 8.3): re-packs new token rows x with the routing of an earlier
  * ep_dispatch whose handle is passed, skipping the layout, the slot
@@ -210,6 +243,24 @@ ep_status_t ep_dispatch_noalloc(const void* x, int32_t T, int32_t H, const int64
  */
 ep_status_t ep_combine(const void* y, const ep_handle_t* handle, const float* topk_weights,
                        void* out, void* stream);
+
+/*
+ * Combine with quantised expert outputs and / or a shared expert (the
+ * combine-side int8 / fp8 of low_latency_combine, "DeepEP communication
+ * library guide v2.1", section 1.3.1 and its API listing; the shared-expert
+ * combine of lmdeploy PR #4783).  For every token t,
+ *   out[t] = bf16_rne( fma chain in k order over the unmasked entries of
+ *                      topk_weights[t,k] * value(row(t,k)) ), starting from
+ *                      shared[t] (bf16) if given, else +0,
+ * where value = the bf16 row (y_quant EP_QUANT_NONE) or, for FP8 e4m3 / int8
+ * codes, decode(code) * scale as an fp32 product with one fp32 scale per
+ * y_quant_size channels (y_scales [recv_capacity, H / y_quant_size]).
+ * y_quant_size: 16..512 (a power of two) or H.  shared may be NULL.  With
+ * y_quant NONE and shared NULL this is ep_combine.
+ */
+ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,
+                          const ep_handle_t* handle, const float* topk_weights, const void* shared, void* out,
+                          void* stream);
 
 /* Waits for `stream`, then copies the device status word to *host_status.
  * Returns EP_OK, or EP_ERR_CUDA if the wait or the copy failed. */
