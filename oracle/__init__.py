@@ -16,7 +16,7 @@ import numpy as np
 from . import build as _build
 
 OK, INVALID_ARG, BAD_EXPERT_ID, CAPACITY = 0, 1, 2, 3
-QUANT = {"none": 0, "fp8": 1, "int8": 2}
+QUANT = {"none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 
 
 class OracleError(RuntimeError):
@@ -61,6 +61,14 @@ def lib():
         L.oracle_ll_slots.restype = C.c_int
         L.oracle_combine_rows_q.argtypes = [p, p, i32, i32, i64, i32, i32, i32, p, p, p, p, i64, p]
         L.oracle_combine_rows_q.restype = C.c_int
+        L.oracle_e2m1_to_f64.argtypes = [C.c_uint8]
+        L.oracle_e2m1_to_f64.restype = C.c_double
+        L.oracle_f32_to_e2m1.argtypes = [C.c_float]
+        L.oracle_f32_to_e2m1.restype = C.c_uint8
+        L.oracle_quantize_row_mx.argtypes = [p, i32, i32, i32, i32, i32, p, p]
+        L.oracle_quantize_row_mx.restype = C.c_int
+        L.oracle_dispatch_rows_mx.argtypes = [p, i32, i32, i32, p, i32, i32, i32, i32, p, i64, p, p, i64]
+        L.oracle_dispatch_rows_mx.restype = C.c_int
         L.oracle_f32_to_e4m3_n.argtypes = [p, i64, p]
         L.oracle_f32_to_e4m3_n.restype = None
         L.oracle_f32_to_bf16_n.argtypes = [p, i64, p]
@@ -301,3 +309,58 @@ def combine_rows_q(y, y_scales, quant: str, quant_size: int, dst_buffer_slot_idx
     if st:
         raise OracleError(st, "combine_rows_q")
     return out
+
+
+# ------------------------------------------------------- MXFP4 and UE8M0
+
+def e2m1_to_f64(codes) -> np.ndarray:
+    f = lib().oracle_e2m1_to_f64
+    return np.array([f(int(c)) for c in np.asarray(codes).ravel()], np.float64).reshape(np.shape(codes))
+
+
+def f32_to_e2m1(x) -> np.ndarray:
+    f = lib().oracle_f32_to_e2m1
+    return np.array([f(float(v)) for v in np.asarray(x, np.float32).ravel()], np.uint8).reshape(np.shape(x))
+
+
+def row_layout(H: int, quant: str, quant_size: int, scale_ue8m0: bool):
+    """(code bytes per row, scale dtype, scales per row) of a received row."""
+    if quant == "none":
+        return 2 * H, None, 0
+    ue8 = scale_ue8m0 or quant == "mxfp4"
+    return (H // 2 if quant == "mxfp4" else H), (np.uint8 if ue8 else np.float32), H // quant_size
+
+
+def quantize_row_mx(x_row, quant: str, quant_size: int, round_scale: bool = False, scale_ue8m0: bool = False):
+    xr = _c(x_row, np.uint16)
+    H = xr.shape[0]
+    nb, sdt, ns = row_layout(H, quant, quant_size, scale_ue8m0)
+    q = np.zeros(nb, np.uint8)
+    sc = np.zeros(ns, sdt)
+    st = lib().oracle_quantize_row_mx(_ptr(xr), H, QUANT[quant], quant_size, int(round_scale), int(scale_ue8m0),
+                                      _ptr(q), _ptr(sc))
+    if st:
+        raise OracleError(st, "quantize_row_mx")
+    return q, sc
+
+
+def dispatch_rows_mx(x, dst_buffer_slot_idx, quant: str, quant_size: int, round_scale: bool = False,
+                     scale_ue8m0: bool = False, tokens=None, num_rows: Optional[int] = None):
+    """recv_x code bytes [rows, row_bytes] and scales [rows, H/quant_size] (fp32 or UE8M0 bytes)."""
+    xs = _c(x, np.uint16)
+    dst = _c(dst_buffer_slot_idx, np.int32)
+    T, H = xs.shape
+    K = dst.shape[1]
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tok = _c(tokens, np.int32)
+    rows = (int(dst.max()) + 1 if dst.size else 0) if num_rows is None else num_rows
+    nb, sdt, ns = row_layout(H, quant, quant_size, scale_ue8m0)
+    recv_x = np.zeros((rows, nb), np.uint8)
+    recv_scales = None if sdt is None else np.zeros((rows, ns), sdt)
+    st = lib().oracle_dispatch_rows_mx(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size, int(round_scale),
+                                       int(scale_ue8m0), _ptr(tok), tok.shape[0], _ptr(recv_x),
+                                       _ptr(recv_scales), rows)
+    if st:
+        raise OracleError(st, "dispatch_rows_mx")
+    return recv_x, recv_scales

@@ -455,3 +455,124 @@ int oracle_combine_rows_q(const void* y, const float* y_scales, int quant, int q
     }
     return OR_OK;
 }
+
+/* ------------------------------------------------ MXFP4 and UE8M0 scales */
+
+#define OR_QUANT_MXFP4 3
+
+/* OCP FP4 E2M1: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit; exponent
+ * field 0 is subnormal (m * 0.5); no infinities or NaN; the largest value is
+ * 1.5 * 2^2 = 6. */
+double oracle_e2m1_to_f64(uint8_t c) {
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* binary32 -> E2M1, round to nearest even, saturating to +-6 (finite input). */
+uint8_t oracle_f32_to_e2m1(float x) {
+    uint8_t sign = signbit(x) ? 8 : 0;
+    double a = fabs((double)x);
+    if (a >= 6.0) return (uint8_t)(sign | 7);
+    if (a == 0.0) return sign;
+    int ex;
+    frexp(a, &ex);
+    int e2 = ex - 1;                                   /* 2^e2 <= a < 2^(e2+1) */
+    double q = (e2 < 0) ? 0.5 : ldexp(1.0, e2 - 1);    /* spacing in the binade */
+    double v = nearbyint(a / q) * q;                   /* nearest, ties even */
+    if (v == 0.0) return sign;
+    if (v < 1.0) return (uint8_t)(sign | 1);           /* 0.5: subnormal */
+    frexp(v, &ex);
+    e2 = ex - 1;
+    int m = (int)((v / ldexp(1.0, e2) - 1.0) * 2.0);   /* 0 or 1 */
+    return (uint8_t)(sign | ((e2 + 1) << 1) | m);
+}
+
+/* Quantises one bf16 row with the scale encodings of the low-latency API:
+ *  - OR_QUANT_FP8 / OR_QUANT_INT8 as oracle_quantize_row; with scale_ue8m0 the
+ *    (power-of-two, round_scale required) scales are stored as one UE8M0 byte
+ *    each: the biased exponent 127 + log2(s) (use_ue8m0 of guide v2.1);
+ *  - OR_QUANT_MXFP4 (quant_size 32, guide v2.1 section 1.3.3): per group of 32
+ *    the OCP MX shared scale X = 2^(floor(log2 amax) - 2) (2 = the largest
+ *    exponent of E2M1; amax floored at 1e-4), elements E2M1(x / X), two per
+ *    byte (even element in the low nibble), scale stored as a UE8M0 byte.
+ * q receives the row's code bytes (H, or H/2 for MXFP4); scales receives
+ * H/quant_size floats or bytes. */
+int oracle_quantize_row_mx(const uint16_t* x, int H, int quant, int quant_size, int round_scale,
+                           int scale_ue8m0, uint8_t* q, void* scales) {
+    if (quant == OR_QUANT_MXFP4) {
+        if (quant_size != 32 || H % 32 != 0) return OR_INVALID_ARG;
+        for (int g = 0; g < H / 32; ++g) {
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float v = fabsf(oracle_bf16_to_f32(x[g * 32 + i]));
+                if (v > amax) amax = v;
+            }
+            if (amax < 1e-4f) amax = 1e-4f;
+            int ex;
+            frexp((double)amax, &ex);
+            int E = (ex - 1) - 2;                        /* floor(log2 amax) - 2 */
+            float s = (float)ldexp(1.0, E);
+            ((uint8_t*)scales)[g] = (uint8_t)(E + 127);
+            for (int i = 0; i < 32; i += 2) {
+                uint8_t lo = oracle_f32_to_e2m1(oracle_bf16_to_f32(x[g * 32 + i]) / s);
+                uint8_t hi = oracle_f32_to_e2m1(oracle_bf16_to_f32(x[g * 32 + i + 1]) / s);
+                q[(g * 32 + i) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+        return OR_OK;
+    }
+    if (!scale_ue8m0) return oracle_quantize_row(x, H, quant, quant_size, round_scale, q, (float*)scales);
+    if (!round_scale) return OR_INVALID_ARG;             /* bytes hold powers of two only */
+    if (quant_size < 1 || H % quant_size != 0) return OR_INVALID_ARG;
+    float* f = malloc(sizeof(float) * (size_t)(H / quant_size));
+    int st = oracle_quantize_row(x, H, quant, quant_size, round_scale, q, f);
+    for (int g = 0; st == OR_OK && g < H / quant_size; ++g) {
+        int ex;
+        double m = frexp((double)f[g], &ex);              /* f = 0.5 * 2^ex exactly */
+        if (m != 0.5) { st = OR_INVALID_ARG; break; }
+        ((uint8_t*)scales)[g] = (uint8_t)((ex - 1) + 127);
+    }
+    free(f);
+    return st;
+}
+
+/* oracle_dispatch_rows for every quantisation, including MXFP4 and UE8M0
+ * scale bytes.  Row bytes: 2H (bf16), H (FP8 / int8), H/2 (MXFP4); scale
+ * bytes per row: H/quant_size times 4 (fp32) or 1 (UE8M0, always for MXFP4). */
+int oracle_dispatch_rows_mx(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
+                            int quant, int quant_size, int round_scale, int scale_ue8m0,
+                            const int32_t* tokens, int64_t n_tokens, uint8_t* recv_x, uint8_t* recv_scales,
+                            int64_t capacity) {
+    if (H < 1) return OR_INVALID_ARG;
+    int ue8 = (quant == OR_QUANT_MXFP4) || scale_ue8m0;
+    int64_t row_bytes = quant == OR_QUANT_NONE ? 2 * (int64_t)H : quant == OR_QUANT_MXFP4 ? H / 2 : H;
+    int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
+    int64_t scale_bytes = (int64_t)ns * (ue8 ? 1 : 4);
+    uint8_t* q = malloc((size_t)H);
+    uint8_t* sc = malloc((size_t)(scale_bytes > 0 ? scale_bytes : 1));
+    int st = OR_OK;
+    for (int64_t i = 0; i < n_tokens && st == OR_OK; ++i) {
+        int t = tokens[i];
+        if (t < 0 || t >= T) { st = OR_INVALID_ARG; break; }
+        const uint16_t* xr = x + (int64_t)t * H;
+        if (quant != OR_QUANT_NONE) {
+            st = oracle_quantize_row_mx(xr, H, quant, quant_size, round_scale, scale_ue8m0, q, sc);
+            if (st) break;
+        }
+        for (int k = 0; k < K; ++k) {
+            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+            if (row < 0) continue;
+            if (row >= capacity) { st = OR_CAPACITY; break; }
+            if (quant == OR_QUANT_NONE) {
+                memcpy(recv_x + row * row_bytes, xr, (size_t)row_bytes);
+            } else {
+                memcpy(recv_x + row * row_bytes, q, (size_t)row_bytes);
+                memcpy(recv_scales + row * scale_bytes, sc, (size_t)scale_bytes);
+            }
+        }
+    }
+    free(q);
+    free(sc);
+    return st;
+}
