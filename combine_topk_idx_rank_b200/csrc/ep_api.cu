@@ -84,6 +84,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
             pa.n_tok_items = R * per_round; pa.do_pad = (j == 0) && !h->low_latency;
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
+            pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
@@ -99,6 +100,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
 // Quantisation options shared by ep_dispatch and ep_dispatch_cached.
 bool quant_ok(int quant, int quant_size, int H, const float* recv_scales) {
     if (quant == EP_QUANT_NONE) return true;
+    if (quant == EP_QUANT_MXFP4) return quant_size == 32 && H % 32 == 0 && recv_scales != nullptr;
     if (quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8) return false;
     const bool group = quant_size == 16 || quant_size == 32 || quant_size == 64 || quant_size == 128 ||
                        quant_size == 256 || quant_size == 512;
@@ -168,6 +170,8 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     if (recv_capacity < 0 || recv_capacity >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
     if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
+        return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
         h->err == nullptr)
         return EP_ERR_INVALID_ARG;
@@ -226,6 +230,8 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
     const int quant = opts->quant;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
     if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
+        return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
         h->err == nullptr || h->recv_src_metadata == nullptr)
         return EP_ERR_INVALID_ARG;
@@ -274,6 +280,8 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
     const int quant = opts->quant;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
     if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
+        return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
         h->err == nullptr)
         return EP_ERR_INVALID_ARG;
@@ -293,6 +301,7 @@ ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant,
     if (!sizes_ok(T, K, h->num_experts, R)) return EP_ERR_INVALID_ARG;
     if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
     if (h->err == nullptr) return EP_ERR_INVALID_ARG;
+    if (y_quant == EP_QUANT_MXFP4) return EP_ERR_INVALID_ARG;   // combine reads FP8 / int8 codes only
     const int qs = y_quant == EP_QUANT_NONE ? 0 : y_quant_size;
     if (!quant_ok(y_quant, qs, H, y_quant == EP_QUANT_NONE ? nullptr : y_scales)) return EP_ERR_INVALID_ARG;
     if (T > 0 && (out == nullptr || topk_weights == nullptr || h->dst_buffer_slot_idx == nullptr))

@@ -113,6 +113,7 @@ struct PackArgs {
     const int32_t* cnt;         // [E] unaligned counts (handle): padding map source
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
+    int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
     int32_t* err;
 };
 

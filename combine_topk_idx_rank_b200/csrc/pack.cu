@@ -19,6 +19,7 @@
 // Quantised rows are computed by threads from 16-byte vector loads and
 // written with 16-byte vector stores.
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "ep_internal.cuh"
@@ -37,7 +38,7 @@ namespace ep {
 
 namespace {
 
-constexpr int kQuantFp8 = 1, kQuantInt8 = 2;
+constexpr int kQuantFp8 = 1, kQuantInt8 = 2, kQuantMxfp4 = 3;
 constexpr int kBulkChunk = 16384;          // max bytes per pipeline stage
 constexpr unsigned kSpinLimit = 1u << 24;  // bounded mbarrier waits
 
@@ -215,6 +216,45 @@ __device__ __forceinline__ float amax16(const float (&f)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(f[i]));
     return m;
+}
+
+// MXFP4 shared scale of a 32-channel group: 2^(floor(log2 amax) - 2), 2 being
+// the largest exponent of E2M1 (the OCP MX conversion); amax floored at 1e-4.
+__device__ __forceinline__ float mx_scale(float amax) {
+    const uint32_t biased = (__float_as_uint(fmaxf(amax, 1e-4f)) >> 23) & 0xffu;
+    return __uint_as_float((biased - 2u) << 23);
+}
+
+// UE8M0 byte of a positive power of two: its biased exponent.
+__device__ __forceinline__ uint8_t ue8m0_of(float s) { return (uint8_t)((__float_as_uint(s) >> 23) & 0xffu); }
+
+// 16 channels -> 16 E2M1 codes, two per byte (even channel in the low nibble).
+__device__ __forceinline__ uint2 quant16_fp4(const float (&f)[16], float s) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        w[h] = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_fp4x2_storage_t b = __nv_cvt_float2_to_fp4x2(
+                make_float2(__fdiv_rn(f[8 * h + 2 * i], s), __fdiv_rn(f[8 * h + 2 * i + 1], s)), __NV_E2M1,
+                cudaRoundNearest);
+            w[h] |= (uint32_t)b << (8 * i);
+        }
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ void store_scale(const PackArgs& a, size_t idx, float s) {
+    if (a.scale_bytes) reinterpret_cast<uint8_t*>(a.recv_scales)[idx] = ue8m0_of(s);
+    else a.recv_scales[idx] = s;
+}
+
+__device__ __forceinline__ void zero_scales(const PackArgs& a, int64_t row, int nscales) {
+    for (int j = threadIdx.x; j < nscales; j += blockDim.x) {
+        if (a.scale_bytes) reinterpret_cast<uint8_t*>(a.recv_scales)[row * nscales + j] = 0;
+        else a.recv_scales[row * nscales + j] = 0.0f;
+    }
 }
 
 __device__ __forceinline__ float finish_scale(float amax, float qmax, int round_scale) {
@@ -402,8 +442,9 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 }
 
 // ------------------------------------------------- group quantisation (<=512)
-// A thread owns 16 consecutive channels (two 16-byte loads, one 16-byte
-// store); a group of G channels is G/16 adjacent lanes, reduced by shuffles.
+// A thread owns 16 consecutive channels (two 16-byte loads; one 16-byte store
+// of FP8 / int8 codes, or one 8-byte store of 16 E2M1 codes); a group of G
+// channels is G/16 adjacent lanes, reduced by shuffles.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
     grid_dependency_wait();
@@ -412,8 +453,10 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
+    constexpr int kUnitBytes = QUANT == kQuantMxfp4 ? 8 : 16;   // code bytes of 16 channels
     const int tid = threadIdx.x;
     const int U = a.H / 16;
+    const size_t row_bytes = (size_t)U * kUnitBytes;
     const int nscales = a.H / G;
     const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     const int n_items = a.n_tok_items + n_pad;
@@ -439,19 +482,29 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
                     float m = amax16(f);
 #pragma unroll
                     for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    sc[j] = finish_scale(m, kQmax, a.round_scale);
-                    q[j] = quant16<QUANT>(f, sc[j]);
+                    if constexpr (QUANT == kQuantMxfp4) {
+                        sc[j] = mx_scale(m);
+                        const uint2 c = quant16_fp4(f, sc[j]);
+                        q[j] = make_uint4(c.x, c.y, 0, 0);
+                    } else {
+                        sc[j] = finish_scale(m, kQmax, a.round_scale);
+                        q[j] = quant16<QUANT>(f, sc[j]);
+                    }
                 }
                 for (int k = 0; k < a.K; ++k) {
                     const int slot = s_slot[k];
                     if (slot < 0) continue;
-                    uint8_t* dst = a.recv_x + (size_t)slot * a.H;
+                    uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
 #pragma unroll
                     for (int j = 0; j < UPT; ++j) {
                         const int u = u0 + j * blockDim.x + tid;
                         if (u < U) {
-                            st_v4(dst + 16 * (size_t)u, q[j]);
-                            if ((u % kLanes) == 0) a.recv_scales[(size_t)slot * nscales + u / kLanes] = sc[j];
+                            if constexpr (QUANT == kQuantMxfp4) {
+                                *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[j].x, q[j].y);
+                            } else {
+                                st_v4(dst + 16 * (size_t)u, q[j]);
+                            }
+                            if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[j]);
                         }
                     }
                 }
@@ -459,9 +512,9 @@ __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
-                uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
-                for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                for (int j = tid; j < nscales; j += blockDim.x) a.recv_scales[(size_t)row * nscales + j] = 0.0f;
+                uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * row_bytes);
+                for (size_t v = tid; v < row_bytes / 16; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
+                zero_scales(a, row, nscales);
             }
         }
         __syncthreads();
@@ -535,14 +588,14 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
                     const int u = j * blockDim.x + tid;
                     if (u < U) st_v4(dst + 16 * (size_t)u, raw[j][0]);
                 }
-                if (tid == 0) a.recv_scales[slot] = sc;
+                if (tid == 0) store_scale(a, (size_t)slot, sc);
             }
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                if (tid == 0) a.recv_scales[row] = 0.0f;
+                if (tid == 0) zero_scales(a, row, 1);
             }
         }
         __syncthreads();
@@ -571,6 +624,10 @@ template <int QUANT>
 cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
     const int U = a.H / 16;
     const int threads = min(256, round_up32((U + 1) / 2));   // 2 units per thread
+    if constexpr (QUANT == kQuantMxfp4) {
+        if (a.quant_size != 32) return cudaErrorInvalidValue;
+        return run(k_pack_group<kQuantMxfp4, 32, 2>, threads, a, st);
+    }
     switch (a.quant_size) {
         case 16: return run(k_pack_group<QUANT, 16, 2>, threads, a, st);
         case 32: return run(k_pack_group<QUANT, 32, 2>, threads, a, st);
@@ -620,6 +677,7 @@ cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st) {
         return launch_bulk(a, st);
 #endif
     }
+    if (quant == EP_QUANT_MXFP4) return launch_group<kQuantMxfp4>(a, st);
     const bool per_token = a.quant_size == a.H;
     if (quant == EP_QUANT_FP8_E4M3)
         return per_token ? launch_token<kQuantFp8>(a, st) : launch_group<kQuantFp8>(a, st);

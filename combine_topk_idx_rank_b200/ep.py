@@ -29,7 +29,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(HERE, "libep.so")
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, EP_ERR_TIMEOUT = range(6)
-_QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2}
+_QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
@@ -44,7 +44,7 @@ class EPError(RuntimeError):
 
 class _Opts(C.Structure):
     _fields_ = [("expert_alignment", C.c_int32), ("quant", C.c_int32), ("quant_size", C.c_int32),
-                ("round_scale", C.c_int32), ("num_rounds", C.c_int32), ("reserved", C.c_int32),
+                ("round_scale", C.c_int32), ("num_rounds", C.c_int32), ("scale_ue8m0", C.c_int32),
                 ("cumulative_local_expert_recv_stats", C.c_void_p),
                 ("event_pack_begin", C.c_void_p), ("event_pack_end", C.c_void_p)]
 
@@ -187,21 +187,31 @@ class DispatchBuffers:
     quant_size: int
 
 
+def _recv_tensors(rows: int, H: int, q: Optional[str], quant_size: int, scale_ue8m0: bool, dev):
+    """recv_x and recv_scales for `rows` received rows: bf16 rows; FP8 e4m3 /
+    int8 codes; or MXFP4 (two E2M1 codes per byte, uint8 [rows, H/2]).  Scales
+    are fp32, or UE8M0 bytes (uint8) with scale_ue8m0 and always for MXFP4."""
+    if q is None:
+        return torch.empty((rows, H), dtype=torch.bfloat16, device=dev), None
+    if q == "mxfp4":
+        return (torch.empty((rows, H // 2), dtype=torch.uint8, device=dev),
+                torch.empty((rows, H // 32), dtype=torch.uint8, device=dev))
+    codes = torch.empty((rows, H), dtype=torch.float8_e4m3fn if q == "fp8" else torch.int8, device=dev)
+    sdt = torch.uint8 if scale_ue8m0 else torch.float32
+    return codes, torch.empty((rows, H // quant_size), dtype=sdt, device=dev)
+
+
 def alloc_dispatch_buffers(num_tokens: int, hidden: int, num_topk: int, num_experts: int,
                            num_ranks: int, expert_alignment: int = 1, quant: Optional[str] = None,
                            quant_size: int = 128, num_rounds: int = 1,
                            recv_capacity: Optional[int] = None,
-                           device: Optional[torch.device] = None) -> DispatchBuffers:
+                           device: Optional[torch.device] = None,
+                           scale_ue8m0: bool = False) -> DispatchBuffers:
     T, H, K, E, R, A = num_tokens, hidden, num_topk, num_experts, num_ranks, expert_alignment
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     cap = recv_capacity_bound(T, K, E, A) if recv_capacity is None else int(recv_capacity)
     q = None if quant in (None, "none") else quant
-    if q is None:
-        recv_x = torch.empty((cap, H), dtype=torch.bfloat16, device=dev)
-        recv_scales = None
-    else:
-        recv_x = torch.empty((cap, H), dtype=torch.float8_e4m3fn if q == "fp8" else torch.int8, device=dev)
-        recv_scales = torch.empty((cap, H // quant_size), dtype=torch.float32, device=dev)
+    recv_x, recv_scales = _recv_tensors(cap, H, q, quant_size, scale_ue8m0, dev)
     i32 = dict(dtype=torch.int32, device=dev)
     handle = EPHandle(T, K, E, R, H, A, num_rounds, cap,
                       topk_idx=torch.empty((T, K), **i32),
@@ -241,17 +251,20 @@ def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: 
     return ntpr, ntpe, itr
 
 
-def _dispatch_cached(x, handle: EPHandle, quant, quant_size, round_scale, num_rounds, buffers, events):
+def _dispatch_cached(x, handle: EPHandle, quant, quant_size, round_scale, num_rounds, buffers, events,
+                     scale_ue8m0=False):
     h = handle
     if tuple(x.shape) != (h.num_tokens, h.hidden):
         raise ValueError("x must be [num_tokens, hidden] of the handle")
     q = None if quant in (None, "none") else quant
     if buffers is None:
         buffers = alloc_dispatch_buffers(h.num_tokens, h.hidden, h.num_topk, h.num_experts, h.num_ranks,
-                                         h.expert_alignment, q, quant_size, num_rounds, h.recv_capacity, x.device)
+                                         h.expert_alignment, q, quant_size, num_rounds, h.recv_capacity, x.device,
+                                         scale_ue8m0)
     if buffers.recv_x.shape[0] != h.recv_capacity:
         raise ValueError("recv_x must have the handle's recv_capacity rows")
-    opts = _Opts(h.expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds, 0,
+    opts = _Opts(h.expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds,
+                 int(bool(scale_ue8m0)),
                  None, None if events is None else events[0].cuda_event,
                  None if events is None else events[1].cuda_event)
     st = _lib.ep_dispatch_cached(_ptr(x), C.byref(h._c()), C.byref(opts), _ptr(buffers.recv_x),
@@ -273,7 +286,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
                 recv_capacity: Optional[int] = None, buffers: Optional[DispatchBuffers] = None,
                 cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
                 layout_out: Optional[tuple] = None, events: Optional[tuple] = None,
-                handle: Optional[EPHandle] = None):
+                handle: Optional[EPHandle] = None, scale_ue8m0: bool = False):
     """Dispatch: returns (recv_x, recv_scales, recv_topk_idx, recv_topk_weights, handle).
 
     With ``do_cpu_sync`` the call waits for the GPU, checks the status word and
@@ -288,7 +301,8 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
     if handle is not None:
         if topk_idx is not None or topk_weights is not None:
             raise ValueError("cached dispatch takes the routing from the handle")
-        return _dispatch_cached(x, handle, quant, quant_size, round_scale, num_rounds, buffers, events)
+        return _dispatch_cached(x, handle, quant, quant_size, round_scale, num_rounds, buffers, events,
+                                scale_ue8m0)
     if topk_idx is None or topk_weights is None or num_experts is None or num_ranks is None:
         raise ValueError("topk_idx, topk_weights, num_experts and num_ranks are required")
     _need_cuda(topk_idx, "topk_idx", torch.int64)
@@ -300,13 +314,16 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
     q = None if quant in (None, "none") else quant
     if q is not None and quant_size not in (16, 32, 64, 128, 256, 512, H):
         raise ValueError(f"quant_size must be a group of 16..512 channels or hidden, got {quant_size}")
+    if q == "mxfp4" and quant_size != 32:
+        raise ValueError("MXFP4 uses groups of 32 channels")
     if buffers is None:
         buffers = alloc_dispatch_buffers(T, H, K, num_experts, num_ranks, expert_alignment, q,
-                                         quant_size, num_rounds, recv_capacity, x.device)
+                                         quant_size, num_rounds, recv_capacity, x.device, scale_ue8m0)
     b = buffers
     h = b.handle
     h.num_rounds = num_rounds
-    opts = _Opts(expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds, 0,
+    opts = _Opts(expert_alignment, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), num_rounds,
+                 int(bool(scale_ue8m0)),
                  None if cumulative_local_expert_recv_stats is None
                  else cumulative_local_expert_recv_stats.data_ptr(),
                  None if events is None else events[0].cuda_event,
@@ -384,7 +401,8 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
                             num_max_dispatch_tokens_per_rank: int, num_experts: int, num_ranks: int,
                             quant: Optional[str] = None, *, quant_size: int = 128, round_scale: bool = False,
                             workspace: Optional[torch.Tensor] = None, buffers: Optional[dict] = None,
-                            cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None):
+                            cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
+                            scale_ue8m0: bool = False):
     """Low-latency (decode) dispatch into fixed-capacity per-expert buffers.
 
     Returns (recv_x [E, R*M, H], recv_scales [E, R*M, H/quant_size] or None,
@@ -404,10 +422,8 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
     b = buffers
     if b is None:
         i32 = dict(dtype=torch.int32, device=dev)
-        b = {"recv_x": torch.empty((rows, H), dtype=(torch.bfloat16 if q is None else
-                                                      torch.float8_e4m3fn if q == "fp8" else torch.int8), device=dev),
-             "recv_scales": None if q is None else torch.empty((rows, H // quant_size), dtype=torch.float32,
-                                                                device=dev),
+        rx, rs = _recv_tensors(rows, H, q, quant_size, scale_ue8m0, dev)
+        b = {"recv_x": rx, "recv_scales": rs,
              "recv_topk_idx": torch.empty((rows, K), **i32),
              "recv_topk_weights": torch.empty((rows, K), dtype=torch.float32, device=dev),
              "count": torch.empty((E,), **i32),
@@ -419,7 +435,7 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
     nbytes = workspace_bytes(T, K, E, R)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
-    opts = _Opts(1, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), 1, 0,
+    opts = _Opts(1, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), 1, int(bool(scale_ue8m0)),
                  None if cumulative_local_expert_recv_stats is None
                  else cumulative_local_expert_recv_stats.data_ptr(), None, None)
     ch = h._c()
@@ -430,5 +446,5 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
     _check(st, "ep_dispatch_low_latency")
     h.recv_capacity, h.low_latency, h.expert_alignment = ch.recv_capacity, 1, 1
     rs = b["recv_scales"]
-    return (b["recv_x"].view(E, R * M, H), None if rs is None else rs.view(E, R * M, -1), b["count"],
+    return (b["recv_x"].view(E, R * M, -1), None if rs is None else rs.view(E, R * M, -1), b["count"],
             b["layout_range"], h)

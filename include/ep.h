@@ -55,7 +55,10 @@ typedef enum {
 typedef enum {
     EP_QUANT_NONE = 0,     /* recv_x is the bf16 row, bit for bit */
     EP_QUANT_FP8_E4M3 = 1, /* OCP e4m3fn codes, fp32 scale per quant_size channels */
-    EP_QUANT_INT8 = 2      /* int8 codes in [-127, 127], fp32 scale per quant_size */
+    EP_QUANT_INT8 = 2,     /* int8 codes in [-127, 127], fp32 scale per quant_size */
+    EP_QUANT_MXFP4 = 3     /* OCP MXFP4: E2M1 codes, two per byte (even channel in the
+                              low nibble), one UE8M0 scale byte per 32 channels
+                              (use_mxfp4, guide v2.1 section 1.3.3) */
 } ep_quant_t;
 
 /* Options of ep_dispatch. */
@@ -65,15 +68,19 @@ typedef struct {
                                  comparative analysis section 3.1) */
     int32_t quant;            /* ep_quant_t */
     int32_t quant_size;       /* channels per scale: 128 (group) or H (per token)
-                                 (quant_size, guide v2.1 section 1.3.1); a multiple
-                                 of 16 that divides H; ignored for EP_QUANT_NONE */
+                                 (quant_size, guide v2.1 section 1.3.1); a power of
+                                 two in [16, 512] dividing H, or H; 32 for MXFP4;
+                                 ignored for EP_QUANT_NONE */
     int32_t round_scale;      /* nonzero: round each scale up to a power of two
                                  (round_scale / use_ue8m0); stored as fp32 */
     int32_t num_rounds;       /* >= 1, divides T / R: the rows are written in
                                  rounds of (T/R)/num_rounds tokens per rank ("ant
                                  moving home" long-sequence mode, Ascend A2 page);
                                  the result equals num_rounds == 1 */
-    int32_t reserved;
+    int32_t scale_ue8m0;      /* nonzero: store each scale as one UE8M0 byte, its
+                                 biased exponent (use_ue8m0, guide v2.1); needs
+                                 round_scale for FP8 / int8; always so for MXFP4.
+                                 recv_scales then points to uint8 [rows, H/quant_size] */
     /* optional device [E]: the unaligned per-expert counts of this call are
      * added to it (cumulative_local_expert_recv_stats, guide v2.1) */
     int32_t* cumulative_local_expert_recv_stats;

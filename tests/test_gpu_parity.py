@@ -268,3 +268,55 @@ def test_cached_dispatch_rejects_routing_args(cuda_device):
     (_, _, _, _, h), _, (x, ti, tw) = gpu_dispatch(cfg, wl, cuda_device)
     with pytest.raises(ValueError):
         ep.ep_dispatch(x, ti, tw, handle=h)
+
+
+@pytest.mark.parametrize("quant,qs,rs,ue8", [("mxfp4", 32, False, False), ("fp8", 128, True, True),
+                                             ("int8", 1024, True, True), ("fp8", 1024, True, True),
+                                             ("int8", 64, True, True)])
+def test_mxfp4_and_ue8m0_scale_bytes(quant, qs, rs, ue8, cuda_device):
+    """MXFP4 (use_mxfp4, groups of 32) and UE8M0 scale bytes (use_ue8m0),
+    bit for bit against the oracle, padding rows included."""
+    cfg = CONFIGS["decode"].scaled(num_tokens=16 * 9, hidden=1024, quant=quant, quant_size=qs, round_scale=rs,
+                                   expert_alignment=4)
+    wl = make_workload(cfg, 0)
+    x, ti, tw = to_dev(wl, cuda_device)
+    recv_x, recv_scales, _, _, h = ep.ep_dispatch(x, ti, tw, 4, quant, num_experts=cfg.num_experts,
+                                                  num_ranks=cfg.num_ranks, quant_size=qs, round_scale=rs,
+                                                  scale_ue8m0=ue8)
+    s = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 4)
+    n = s["num_recv_rows"]
+    assert h.num_recv_rows == n
+    ref_x, ref_s = oracle.dispatch_rows_mx(wl.x, s["dst_buffer_slot_idx"], quant, qs, rs, ue8, num_rows=n)
+    got_x = recv_x.contiguous().view(torch.uint8).cpu().numpy().reshape(n, -1)
+    assert np.array_equal(got_x, ref_x)
+    got_s = recv_scales.contiguous().cpu().numpy()
+    assert got_s.dtype == ref_s.dtype
+    assert np.array_equal(got_s.view(np.uint8), ref_s.view(np.uint8))
+
+
+def test_e2m1_conversion_over_bf16(cuda_device):
+    """Every bf16 value |v| <= 6 through the MXFP4 path with the group scale
+    pinned to 1 (each 32-group also holds 4.0, so floor(log2 amax) - 2 = 0)."""
+    allv = (np.arange(0, 0x7f80, dtype=np.uint32) << 16).view(np.float32)
+    v = allv[allv <= 6.0]
+    v = np.concatenate([v, -v]).astype(np.float32)
+    per = 31
+    ng = -(-v.size // per)
+    v = np.concatenate([v, np.zeros(ng * per - v.size, np.float32)]).reshape(ng, per)
+    g = np.concatenate([np.full((ng, 1), 4.0, np.float32), v], axis=1)
+    H, R = 1024, 8
+    T = -(-(-(-ng * 32 // H)) // R) * R
+    flat = np.full(T * H, 4.0, np.float32)
+    flat[:g.size] = g.ravel()
+    cfg = CONFIGS["tiny"].scaled(num_tokens=T, hidden=H, quant="mxfp4", quant_size=32)
+    wl = make_workload(cfg, 0)
+    wl.x = torch.from_numpy(flat.reshape(T, H)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    x, ti, tw = to_dev(wl, cuda_device)
+    recv_x, recv_scales, _, _, h = ep.ep_dispatch(x, ti, tw, 1, "mxfp4", num_experts=cfg.num_experts,
+                                                  num_ranks=cfg.num_ranks, quant_size=32)
+    s = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks)
+    ref_x, ref_s = oracle.dispatch_rows_mx(wl.x, s["dst_buffer_slot_idx"], "mxfp4", 32,
+                                           num_rows=s["num_recv_rows"])
+    assert np.all(ref_s == 127)
+    assert np.array_equal(recv_x.cpu().numpy(), ref_x)
+    assert np.array_equal(recv_scales.cpu().numpy(), ref_s)
