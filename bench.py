@@ -68,7 +68,7 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(cfg, counts, T):
+def algorithmic_bytes(cfg, counts, T, scale_ue8m0=False, combine_quant=False, low_latency=False):
     """Minimum HBM bytes of one dispatch and one combine, from the actual counts.
 
     Dispatch: topk_idx read once, topk_weights read, x read once, every received
@@ -79,12 +79,16 @@ def algorithmic_bytes(cfg, counts, T):
     H, K, A, E = cfg.hidden, cfg.num_topk, cfg.expert_alignment, cfg.num_experts
     counts = np.asarray(counts, np.int64)
     n = int(counts.sum())
-    n_al = int((-(-counts // A) * A).sum())
-    esize = 2 if cfg.quant == "none" else 1
+    n_al = n if low_latency else int((-(-counts // A) * A).sum())
+    esize = {"none": 2.0, "fp8": 1.0, "int8": 1.0, "mxfp4": 0.5}[cfg.quant]
     nscales = 0 if cfg.quant == "none" else H // cfg.quant_size
-    pack = T * H * 2 + n_al * H * esize + n_al * nscales * 4 + n_al * (2 * K * 4 + 8) + T * K * (8 + 4 + 4)
+    sbytes = 1 if (scale_ue8m0 or cfg.quant == "mxfp4") else 4
+    pack = int(T * H * 2 + n_al * H * esize + n_al * nscales * sbytes + n_al * (2 * K * 4 + 8) + T * K * (8 + 4 + 4))
     layout = T * K * 8 + 4 * E * 4
-    combine = T * K * 8 + n * H * 2 + T * H * 2
+    if combine_quant:       # y rows read as 1-byte codes with fp32 scales
+        combine = T * K * 8 + n * (H + nscales * 4) + T * H * 2
+    else:
+        combine = T * K * 8 + n * H * 2 + T * H * 2
     return {"layout": layout, "pack": pack, "combine": combine, "rows": n, "rows_aligned": n_al}
 
 
@@ -166,12 +170,21 @@ class ClockSampler:
 
 
 def workload_config(args):
-    """The named workload, optionally with a different token count (--tokens)."""
+    """The named workload, optionally with a different token count (--tokens)
+    or dispatch quantisation (--quant, --ue8m0)."""
     cfg = CONFIGS[args.workload]
     if getattr(args, "tokens", 0):
         if args.tokens % (cfg.num_ranks * cfg.num_rounds):
             raise SystemExit(f"--tokens must be a multiple of ranks x rounds = {cfg.num_ranks * cfg.num_rounds}")
         cfg = cfg.scaled(num_tokens=args.tokens)
+    quant = getattr(args, "quant", None)
+    if quant:
+        qs = 32 if quant == "mxfp4" else (cfg.quant_size if cfg.quant != "none" else 128)
+        cfg = cfg.scaled(quant=quant, quant_size=qs)
+    if getattr(args, "ue8m0", False):
+        if cfg.quant not in ("fp8", "int8"):
+            raise SystemExit("--ue8m0 applies to FP8 / int8 dispatch")
+        cfg = cfg.scaled(round_scale=True)
     return cfg
 
 
@@ -247,13 +260,30 @@ def run_ours(args):
     ti = torch.from_numpy(wl.topk_idx).to(dev)
     tw = torch.from_numpy(wl.topk_weights).to(dev)
     q = None if cfg.quant == "none" else cfg.quant
+    ue8 = bool(args.ue8m0)
+    if args.combine_quant and (q not in ("fp8", "int8") or ue8):
+        raise SystemExit("--combine-quant reads FP8 / int8 received rows with fp32 scales")
+    ll = args.mode == "ll"
+    M = T // R                                  # low-latency capacity per (expert, source rank)
     bufs = ep.alloc_dispatch_buffers(T, H, K, E, R, cfg.expert_alignment, q, cfg.quant_size,
-                                     cfg.num_rounds, device=dev)
+                                     cfg.num_rounds, recv_capacity=(E * R * M if ll else None), device=dev,
+                                     scale_ue8m0=ue8)
+    if ll:
+        if cfg.expert_alignment != 1 or cfg.num_rounds != 1:
+            raise SystemExit("--mode ll needs expert_alignment 1 and one round")
+        bufs.handle.low_latency = 1
+        ll_bufs = {"recv_x": bufs.recv_x, "recv_scales": bufs.recv_scales, "recv_topk_idx": bufs.recv_topk_idx,
+                   "recv_topk_weights": bufs.recv_topk_weights,
+                   "count": torch.empty((E,), dtype=torch.int32, device=dev),
+                   "layout_range": torch.empty((E, R), dtype=torch.int64, device=dev), "handle": bufs.handle}
     cap = bufs.recv_x.shape[0]
-    g = torch.Generator(device=dev)
-    g.manual_seed(1234 + rank)
-    y = torch.randn((cap, H), generator=g, device=dev, dtype=torch.bfloat16)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if args.combine_quant:
+        y, y_scales = bufs.recv_x, bufs.recv_scales      # quantised expert outputs (identity experts)
+    else:
+        g = torch.Generator(device=dev)
+        g.manual_seed(1234 + rank)
+        y, y_scales = torch.randn((cap, H), generator=g, device=dev, dtype=torch.bfloat16), None
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for row in ev:               # create the events before handing them to the library
@@ -266,18 +296,30 @@ def run_ours(args):
                        quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
                        do_cpu_sync=False, buffers=bufs)
 
-    def step(i=None):
+    def step(i=None, x=x, ti=ti, tw=tw):
         evs = None if i is None else (ev[i][0], ev[i][1])
         if args.mode == "cached":
             ep.ep_dispatch(x, quant=q, quant_size=cfg.quant_size, round_scale=cfg.round_scale,
-                           num_rounds=cfg.num_rounds, buffers=bufs, events=evs, handle=bufs.handle)
+                           num_rounds=cfg.num_rounds, buffers=bufs, events=evs, handle=bufs.handle,
+                           scale_ue8m0=ue8)
+        elif ll:
+            if evs is not None:
+                evs[0].record()
+            ep.ep_dispatch_low_latency(x, ti, tw, M, E, R, q, quant_size=cfg.quant_size,
+                                       round_scale=cfg.round_scale, workspace=bufs.workspace, buffers=ll_bufs,
+                                       scale_ue8m0=ue8)
+            if evs is not None:
+                evs[1].record()
         else:
             ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
                            quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
-                           do_cpu_sync=False, buffers=bufs, events=evs)
+                           do_cpu_sync=False, buffers=bufs, events=evs, scale_ue8m0=ue8)
         if i is not None:
             ev[i][2].record()
-        ep.ep_combine(y, bufs.handle, tw, out=out)
+        # y: the experts' outputs, produced on the device (random bf16, or the
+        # received codes themselves with --combine-quant)
+        ep.ep_combine(y, bufs.handle, tw, out=out, y_scales=y_scales, quant_size=cfg.quant_size)
+        return out
         if i is not None:
             ev[i][3].record()
 
@@ -318,14 +360,11 @@ def run_ours(args):
     hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
 
     def e2e_step():
+        # the step of the timed loop, from pinned host inputs to the host copy of the result
         dx = hx.to(dev, non_blocking=True)
         dti = hti.to(dev, non_blocking=True)
         dtw = htw.to(dev, non_blocking=True)
-        rx, rs, _, _, h = ep.ep_dispatch(dx, dti, dtw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
-                                         quant_size=cfg.quant_size, round_scale=cfg.round_scale,
-                                         num_rounds=cfg.num_rounds, do_cpu_sync=False, buffers=bufs)
-        yy = rx if q is None else y      # identity experts where recv_x is bf16
-        o = ep.ep_combine(yy, h, dtw, out=out)
+        o = step(None, dx, dti, dtw)
         hout.copy_(o, non_blocking=True)
 
     for _ in range(2):
@@ -343,7 +382,7 @@ def run_ours(args):
     h2d = hx.numel() * 2 + hti.numel() * 8 + htw.numel() * 4
     d2h = hout.numel() * 2
 
-    ab = algorithmic_bytes(cfg, counts, T)
+    ab = algorithmic_bytes(cfg, counts, T, ue8, args.combine_quant, ll)
     if args.mode == "cached":
         ab["layout"] = 0
         ab["pack"] -= T * cfg.num_topk * 8 + ab["rows_aligned"] * (2 * cfg.num_topk * 4 + 8)   # no routing / metadata
@@ -368,7 +407,10 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q is None else f"bf16->{q}",
         "data": "synthetic (seeded numpy PCG64; no dataset, no weights)",
         "config": {"workload": WORKLOAD_DESC[args.workload] + (f" (scaled to {T} tokens)" if args.tokens else "")
-                   + (" — cached dispatch (routing reused from the handle)" if args.mode == "cached" else ""),
+                   + (" — cached dispatch (routing reused from the handle)" if args.mode == "cached" else "")
+                   + (" — low-latency fixed-capacity layout" if ll else "")
+                   + (f" — dispatch {cfg.quant} g{cfg.quant_size}{' ue8m0 bytes' if ue8 else ''}" if args.quant or ue8 else "")
+                   + (" — combine reads the quantised rows" if args.combine_quant else ""),
                    "name": args.workload, "mode": args.mode, "tokens": T, "hidden": H,
                    "num_experts": E, "num_ranks": R, "topk": K, "expert_alignment": cfg.expert_alignment,
                    "quant": cfg.quant, "num_rounds": cfg.num_rounds, "parallelism": f"{world} independent EP problems",
@@ -503,8 +545,14 @@ def main(argv=None):
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--tokens", type=int, default=0, help="scale the workload to this many tokens")
-    p.add_argument("--mode", default="full", choices=["full", "cached"],
-                   help="cached: time dispatch re-packing with a handle (routing computed once)")
+    p.add_argument("--mode", default="full", choices=["full", "cached", "ll"],
+                   help="cached: dispatch re-packing with a handle (routing computed once); "
+                        "ll: low-latency fixed-capacity layout")
+    p.add_argument("--quant", default=None, choices=["none", "fp8", "int8", "mxfp4"],
+                   help="override the workload's dispatch quantisation")
+    p.add_argument("--ue8m0", action="store_true", help="power-of-two scales stored as UE8M0 bytes")
+    p.add_argument("--combine-quant", action="store_true",
+                   help="combine reads the FP8 / int8 received rows (identity experts) instead of bf16 y")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the cpu_baseline sample")
     p.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the --impl reference run")
     p.add_argument("--no-cpu-baseline", action="store_true")
