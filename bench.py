@@ -319,9 +319,9 @@ def run_ours(args):
         # y: the experts' outputs, produced on the device (random bf16, or the
         # received codes themselves with --combine-quant)
         ep.ep_combine(y, bufs.handle, tw, out=out, y_scales=y_scales, quant_size=cfg.quant_size)
-        return out
         if i is not None:
             ev[i][3].record()
+        return out
 
     sampler = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)
                            if str(torch.cuda.get_device_properties(dev).uuid).startswith("GPU-")

@@ -24,9 +24,8 @@
 
 namespace ep {
 
-// YQ: 0 = bf16 expert outputs; 1 = FP8 e4m3 codes, 2 = int8 codes, each value
-// decode(code) * scale (fp32 product) with one fp32 scale per quant_size
-// channels.  With a shared-expert row the accumulator starts from it.
+// Eight codes -> decode(code) * scale (fp32 product).  YQ 1 = FP8 e4m3
+// (decoded exactly through fp16), 2 = int8.
 template <int YQ>
 __device__ __forceinline__ void dequant8(uint2 c, float s, float (&v)[8]) {
     const uint32_t w[2] = {c.x, c.y};
@@ -50,7 +49,7 @@ __device__ __forceinline__ void dequant8(uint2 c, float s, float (&v)[8]) {
     for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], s);
 }
 
-template <int KMAX, int VPT, int YQ>
+template <int KMAX, int VPT>
 __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
@@ -59,7 +58,6 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
     __shared__ int s_n;
     const int tid = threadIdx.x, lane = tid & 31;
     const int V = a.H / 8;                              // slots of 8 channels per row
-    const int nscales = YQ ? a.H / a.quant_size : 0;
     for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
         const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
         if (tid < 32) {
@@ -87,24 +85,14 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
         for (int v0 = 0; v0 < V; v0 += VPT * blockDim.x) {
             // every load of the pass is issued before the first FMA
             uint4 r[VPT][KMAX];
-            uint2 q[VPT][KMAX];
-            float sc[VPT][KMAX];
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
                 if (j < n) {
+                    const uint16_t* yr = reinterpret_cast<const uint16_t*>(a.y) + (size_t)s_slot[j] * a.H;
 #pragma unroll
                     for (int u = 0; u < VPT; ++u) {
                         const int v = v0 + u * blockDim.x + tid;
-                        if (v < V) {
-                            if constexpr (YQ == 0) {
-                                const uint16_t* yr = reinterpret_cast<const uint16_t*>(a.y) + (size_t)s_slot[j] * a.H;
-                                r[u][j] = ld_nc_v4(reinterpret_cast<const uint4*>(yr) + v);
-                            } else {
-                                const uint8_t* yr = reinterpret_cast<const uint8_t*>(a.y) + (size_t)s_slot[j] * a.H;
-                                q[u][j] = __ldg(reinterpret_cast<const uint2*>(yr) + v);
-                                sc[u][j] = __ldg(a.y_scales + (size_t)s_slot[j] * nscales + (v * 8) / a.quant_size);
-                            }
-                        }
+                        if (v < V) r[u][j] = ld_nc_v4(reinterpret_cast<const uint4*>(yr) + v);
                     }
                 }
             }
@@ -125,13 +113,9 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
                     if (j < n) {
                         const float w = s_w[j];
                         float y[8];
-                        if constexpr (YQ == 0) {
-                            const uint4 b = r[u][j];
-                            y[0] = bf16lo(b.x); y[1] = bf16hi(b.x); y[2] = bf16lo(b.y); y[3] = bf16hi(b.y);
-                            y[4] = bf16lo(b.z); y[5] = bf16hi(b.z); y[6] = bf16lo(b.w); y[7] = bf16hi(b.w);
-                        } else {
-                            dequant8<YQ>(q[u][j], sc[u][j], y);
-                        }
+                        const uint4 b = r[u][j];
+                        y[0] = bf16lo(b.x); y[1] = bf16hi(b.x); y[2] = bf16lo(b.y); y[3] = bf16hi(b.y);
+                        y[4] = bf16lo(b.z); y[5] = bf16hi(b.z); y[6] = bf16lo(b.w); y[7] = bf16hi(b.w);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, y[i], acc[i]);
                     }
@@ -154,6 +138,96 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
     }
 }
 
+// Combine of quantised expert outputs: a thread slot covers 16 channels, so
+// each (row, slot) is one 16-byte load of codes and one scale load; all K
+// loads of a slot are issued before the first FMA.
+template <int KMAX, int YQ>
+__global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine_q(CombineArgs a) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+    __shared__ int s_slot[kMaxTopk];
+    __shared__ float s_w[kMaxTopk];
+    __shared__ int s_n;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int V = a.H / 16;                             // slots of 16 channels per row
+    const int nscales = a.H / a.quant_size;
+    const uint8_t* ybase = reinterpret_cast<const uint8_t*>(a.y);
+    for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+        const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
+        if (tid < 32) {
+            int slot = -1;
+            float w = 0.0f;
+            if (lane < a.K) {
+                slot = a.dst_slot[(int64_t)t * a.K + lane];
+                w = a.topk_weights[(int64_t)t * a.K + lane];
+                if (slot >= a.y_rows) {
+                    set_error(a.err, EP_ERR_CAPACITY);
+                    slot = -1;
+                }
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, slot >= 0);
+            if (slot >= 0) {
+                const int pos = __popc(m & lanemask_lt());
+                s_slot[pos] = slot;
+                s_w[pos] = w;
+            }
+            if (lane == 0) s_n = __popc(m);
+        }
+        __syncthreads();
+        const int n = s_n;
+        uint16_t* orow = a.out + (size_t)t * a.H;
+        for (int v = tid; v < V; v += blockDim.x) {
+            uint4 q[KMAX];
+            float sc[KMAX];
+            const int g = (v * 16) / a.quant_size;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < n) {
+                    q[j] = ld_nc_v4(ybase + (size_t)s_slot[j] * a.H + 16 * (size_t)v);
+                    sc[j] = __ldg(a.y_scales + (size_t)s_slot[j] * nscales + g);
+                }
+            }
+            float acc[16];
+            if (a.shared != nullptr) {
+                const uint4* sh = reinterpret_cast<const uint4*>(a.shared + (size_t)t * a.H + 16 * (size_t)v);
+                const uint4 b0 = ld_nc_v4(sh), b1 = ld_nc_v4(sh + 1);
+                const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    acc[2 * i] = bf16lo(w[i]);
+                    acc[2 * i + 1] = bf16hi(w[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < n) {
+                    const float w = s_w[j];
+                    float lo[8], hi[8];
+                    dequant8<YQ>(make_uint2(q[j].x, q[j].y), sc[j], lo);
+                    dequant8<YQ>(make_uint2(q[j].z, q[j].w), sc[j], hi);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[i] = __fmaf_rn(w, lo[i], acc[i]);
+                        acc[8 + i] = __fmaf_rn(w, hi[i], acc[8 + i]);
+                    }
+                }
+            }
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                o[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1])) << 16);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 16 * (size_t)v);
+            st_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            st_v4(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+        }
+        __syncthreads();
+    }
+}
+
 namespace {
 
 template <typename Kern>
@@ -169,22 +243,23 @@ cudaError_t run(Kern k, int threads, const CombineArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
+    if (a.y_quant != EP_QUANT_NONE) {
+        // one 16-channel slot per thread per pass; split the row into equal passes
+        const int V16 = a.H / 16;
+        const int p16 = (V16 + 255) / 256;
+        const int th16 = min(256, ((V16 + p16 - 1) / p16 + 31) & ~31);
+        if (a.y_quant == EP_QUANT_FP8_E4M3)
+            return a.K <= 8 ? run(k_combine_q<8, 1>, th16, a, st) : run(k_combine_q<16, 1>, th16, a, st);
+        return a.K <= 8 ? run(k_combine_q<8, 2>, th16, a, st) : run(k_combine_q<16, 2>, th16, a, st);
+    }
     const int V = a.H / 8;
     // 2 vectors per thread per pass; split the row into equal passes
     const int passes = (V + 2 * 256 - 1) / (2 * 256);
     const int threads = min(256, ((V + 2 * passes - 1) / (2 * passes) + 31) & ~31);
-    if (a.y_quant == EP_QUANT_FP8_E4M3) {
-        if (a.K <= 8) return run(k_combine<8, 2, 1>, threads, a, st);
-        return run(k_combine<16, 1, 1>, threads, a, st);
-    }
-    if (a.y_quant == EP_QUANT_INT8) {
-        if (a.K <= 8) return run(k_combine<8, 2, 2>, threads, a, st);
-        return run(k_combine<16, 1, 2>, threads, a, st);
-    }
-    if (a.K <= 2) return run(k_combine<2, 2, 0>, threads, a, st);
-    if (a.K <= 4) return run(k_combine<4, 2, 0>, threads, a, st);
-    if (a.K <= 8) return run(k_combine<8, EP_COMBINE_VPT, 0>, threads, a, st);
-    return run(k_combine<16, 1, 0>, threads, a, st);
+    if (a.K <= 2) return run(k_combine<2, 2>, threads, a, st);
+    if (a.K <= 4) return run(k_combine<4, 2>, threads, a, st);
+    if (a.K <= 8) return run(k_combine<8, EP_COMBINE_VPT>, threads, a, st);
+    return run(k_combine<16, 1>, threads, a, st);
 }
 
 }  // namespace ep
