@@ -82,7 +82,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.capacity = recv_capacity;
             pa.psum = h->psum_num_recv_tokens_per_expert; pa.cnt = h->num_recv_tokens_per_expert;
             pa.tokens_per_rank = tpr; pa.per_round = per_round; pa.round = j;
-            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0) && !h->low_latency;
+            pa.n_tok_items = R * per_round; pa.do_pad = (j == 0) && !h->low_latency && h->expert_alignment > 1;   // A = 1: no padding rows
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;

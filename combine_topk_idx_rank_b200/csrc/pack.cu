@@ -30,6 +30,9 @@
 #ifndef EP_PACK_LOAD_HINT
 #define EP_PACK_LOAD_HINT 0    // 1: bulk loads of x rows carry an L2 evict-first policy
 #endif
+#ifndef EP_PACK_IEEE_DIV
+#define EP_PACK_IEEE_DIV 0     // 1: every quotient x / scale by the IEEE division
+#endif
 #ifndef EP_PACK_STORE_HINT
 #define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
 #endif
@@ -176,32 +179,63 @@ __device__ __forceinline__ float pow2_ceil_bits(float s) {
     return __uint_as_float(bumped);
 }
 
-template <int QUANT>
-__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float s) {
-    if constexpr (QUANT == kQuantFp8) {
-        const __nv_fp8x2_storage_t lo =
-            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(a, s), __fdiv_rn(b, s)), __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t hi =
-            __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(c, s), __fdiv_rn(d, s)), __NV_SATFINITE, __NV_E4M3);
-        return (uint32_t)lo | ((uint32_t)hi << 16);
-    } else {
-        const int qa = max(-127, min(127, __float2int_rn(__fdiv_rn(a, s))));
-        const int qb = max(-127, min(127, __float2int_rn(__fdiv_rn(b, s))));
-        const int qc = max(-127, min(127, __float2int_rn(__fdiv_rn(c, s))));
-        const int qd = max(-127, min(127, __float2int_rn(__fdiv_rn(d, s))));
-        return (uint32_t)(qa & 0xff) | ((uint32_t)(qb & 0xff) << 8) | ((uint32_t)(qc & 0xff) << 16) |
-               ((uint32_t)(qd & 0xff) << 24);
+// Quotients x / s rounded to nearest even.  With r = RN(1/s), y = RN(x r) is
+// within one ulp of x / s, the remainder x - s y is exact in one fused
+// multiply-add, and the corrected y + r (x - s y) rounds to RN(x / s)
+// (Markstein's theorem on division with a fused multiply-add, IBM J. Res.
+// Develop. 34(1), 1990) -- provided nothing underflows: x and x / s must stay
+// well above the smallest normal.  So the corrected product is used when all
+// 16 inputs satisfy |x| >= max(2^-100, 2^-100 s); otherwise (a zero, a tiny
+// value, a NaN, or an infinite s) all 16 take the IEEE division.  Over every
+// pair of a bf16 x and a bf16 group maximum (scale = max(amax, 1e-4) / 448 or
+// / 127), the rule gives the same bits as the IEEE division.
+template <bool FAST>
+__device__ __forceinline__ void divide16(const float (&f)[16], float s, float (&v)[16]) {
+    if constexpr (!FAST || EP_PACK_IEEE_DIV) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(f[i], s);
+        return;
+    }
+    const float floor_ = fmaxf(0x1p-100f, __fmul_rn(0x1p-100f, s));
+    const float r = __frcp_rn(s);
+    bool fast = true;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        fast &= fabsf(f[i]) >= floor_;
+        const float y = __fmul_rn(f[i], r);
+        v[i] = __fmaf_rn(__fmaf_rn(-y, s, f[i]), r, y);
+    }
+    if (!fast) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(f[i], s);
     }
 }
 
-template <int QUANT>
+// 16 channels -> 16 FP8 e4m3 (RNE, saturating) or int8 (RNE, clamped to
+// +-127) codes of x / s.  FAST: quotients by the rule of divide16 (the
+// per-token kernel, capped at 64 registers, keeps the plain IEEE division).
+template <int QUANT, bool FAST = true>
 __device__ __forceinline__ uint4 quant16(const float (&f)[16], float s) {
-    uint4 q;
-    q.x = quant4<QUANT>(f[0], f[1], f[2], f[3], s);
-    q.y = quant4<QUANT>(f[4], f[5], f[6], f[7], s);
-    q.z = quant4<QUANT>(f[8], f[9], f[10], f[11], s);
-    q.w = quant4<QUANT>(f[12], f[13], f[14], f[15], s);
-    return q;
+    float v[16];
+    divide16<FAST>(f, s, v);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (QUANT == kQuantFp8) {
+            const __nv_fp8x2_storage_t lo =
+                __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i], v[4 * i + 1]), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t hi =
+                __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2], v[4 * i + 3]), __NV_SATFINITE, __NV_E4M3);
+            w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+        } else {
+            uint32_t b = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                b |= (uint32_t)(max(-127, min(127, __float2int_rn(v[4 * i + j]))) & 0xff) << (8 * j);
+            w[i] = b;
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ void unpack16(uint4 lo, uint4 hi, float (&f)[16]) {
@@ -230,6 +264,8 @@ __device__ __forceinline__ uint8_t ue8m0_of(float s) { return (uint8_t)((__float
 
 // 16 channels -> 16 E2M1 codes, two per byte (even channel in the low nibble).
 __device__ __forceinline__ uint2 quant16_fp4(const float (&f)[16], float s) {
+    float v[16];
+    divide16<true>(f, s, v);
     uint32_t w[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -237,8 +273,7 @@ __device__ __forceinline__ uint2 quant16_fp4(const float (&f)[16], float s) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const __nv_fp4x2_storage_t b = __nv_cvt_float2_to_fp4x2(
-                make_float2(__fdiv_rn(f[8 * h + 2 * i], s), __fdiv_rn(f[8 * h + 2 * i + 1], s)), __NV_E2M1,
-                cudaRoundNearest);
+                make_float2(v[8 * h + 2 * i], v[8 * h + 2 * i + 1]), __NV_E2M1, cudaRoundNearest);
             w[h] |= (uint32_t)b << (8 * i);
         }
     }
@@ -442,81 +477,126 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 }
 
 // ------------------------------------------------- group quantisation (<=512)
-// A thread owns 16 consecutive channels (two 16-byte loads; one 16-byte store
-// of FP8 / int8 codes, or one 8-byte store of 16 E2M1 codes); a group of G
-// channels is G/16 adjacent lanes, reduced by shuffles.
+// A thread owns 16 consecutive channels per unit (two 16-byte loads; one
+// 16-byte store of FP8 / int8 codes, or one 8-byte store of 16 E2M1 codes); a
+// group of G channels is G/16 adjacent lanes, reduced by shuffles.  A work
+// item is one pass (UPT x blockDim units) over one token's row, or one padding
+// row.  The CTA's next item is fetched (its x units into registers, its
+// destination rows into the other half of s_slot) before the current item is
+// quantised and stored, so its loads are in flight during that work.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
-    __shared__ int s_slot[kMaxTopk];
+    __shared__ int s_slot[2][kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     constexpr int kUnitBytes = QUANT == kQuantMxfp4 ? 8 : 16;   // code bytes of 16 channels
     const int tid = threadIdx.x;
     const int U = a.H / 16;
+    const int per_pass = UPT * blockDim.x;
+    const int passes = (U + per_pass - 1) / per_pass;
     const size_t row_bytes = (size_t)U * kUnitBytes;
     const int nscales = a.H / G;
     const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
-    const int n_items = a.n_tok_items + n_pad;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        if (item < a.n_tok_items) {
-            const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
-            load_slots(a, t, s_slot);
-            __syncthreads();
-            const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
-            for (int u0 = 0; u0 < U; u0 += UPT * blockDim.x) {
-                uint4 q[UPT];
-                float sc[UPT];
+    const int n_tok = a.n_tok_items * passes;
+    const int n_items = n_tok + n_pad;
+
+    // item -> token, and the first unit of its pass
+    auto locate = [&](int item, int& t, int& u0) {
+        const int ti = item / passes;
+        u0 = (item - ti * passes) * per_pass;
+        t = token_of_item(ti, a.tokens_per_rank, a.per_round, a.round);
+    };
+    // issues the loads of a token item: its units into r, its rows into slot
+    auto fetch = [&](int item, uint4 (&r)[UPT][2], int& slot) {
+        int t, u0;
+        locate(item, t, u0);
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
+#pragma unroll
+        for (int j = 0; j < UPT; ++j) {
+            const int u = u0 + j * blockDim.x + tid;
+            if (u < U) {
+                r[j][0] = ld_nc_v4(xr + 2 * u);
+                r[j][1] = ld_nc_v4(xr + 2 * u + 1);
+            } else {
+                r[j][0] = r[j][1] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        slot = tid < a.K ? a.dst_slot[(int64_t)t * a.K + tid] : -1;
+    };
+
+    uint4 raw[UPT][2];
+    int slot_next = -1;
+    int item = blockIdx.x;
+    if (item < n_tok) fetch(item, raw, slot_next);
+    if (tid < a.K) s_slot[0][tid] = slot_next;
+    __syncthreads();
+    int buf = 0;
+    for (; item < n_items; item += gridDim.x) {
+        const int nxt = item + gridDim.x;
+        uint4 nraw[UPT][2];
+        slot_next = -1;
+        if (nxt < n_tok) {
+            fetch(nxt, nraw, slot_next);
+        } else {
+#pragma unroll
+            for (int j = 0; j < UPT; ++j) nraw[j][0] = nraw[j][1] = make_uint4(0, 0, 0, 0);
+        }
+        if (item < n_tok) {
+            int t, u0;
+            locate(item, t, u0);
+            uint4 q[UPT];
+            float sc[UPT];
+#pragma unroll
+            for (int j = 0; j < UPT; ++j) {
+                float f[16];
+                unpack16(raw[j][0], raw[j][1], f);
+                float m = amax16(f);
+#pragma unroll
+                for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if constexpr (QUANT == kQuantMxfp4) {
+                    sc[j] = mx_scale(m);
+                    const uint2 c = quant16_fp4(f, sc[j]);
+                    q[j] = make_uint4(c.x, c.y, 0, 0);
+                } else {
+                    sc[j] = finish_scale(m, kQmax, a.round_scale);
+                    q[j] = quant16<QUANT>(f, sc[j]);
+                }
+            }
+            for (int k = 0; k < a.K; ++k) {
+                const int slot = s_slot[buf][k];
+                if (slot < 0) continue;
+                uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
                     const int u = u0 + j * blockDim.x + tid;
-                    float f[16];
                     if (u < U) {
-                        unpack16(ld_nc_v4(xr + 2 * u), ld_nc_v4(xr + 2 * u + 1), f);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) f[i] = 0.0f;
-                    }
-                    float m = amax16(f);
-#pragma unroll
-                    for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    if constexpr (QUANT == kQuantMxfp4) {
-                        sc[j] = mx_scale(m);
-                        const uint2 c = quant16_fp4(f, sc[j]);
-                        q[j] = make_uint4(c.x, c.y, 0, 0);
-                    } else {
-                        sc[j] = finish_scale(m, kQmax, a.round_scale);
-                        q[j] = quant16<QUANT>(f, sc[j]);
-                    }
-                }
-                for (int k = 0; k < a.K; ++k) {
-                    const int slot = s_slot[k];
-                    if (slot < 0) continue;
-                    uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
-#pragma unroll
-                    for (int j = 0; j < UPT; ++j) {
-                        const int u = u0 + j * blockDim.x + tid;
-                        if (u < U) {
-                            if constexpr (QUANT == kQuantMxfp4) {
-                                *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[j].x, q[j].y);
-                            } else {
-                                st_v4(dst + 16 * (size_t)u, q[j]);
-                            }
-                            if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[j]);
+                        if constexpr (QUANT == kQuantMxfp4) {
+                            *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[j].x, q[j].y);
+                        } else {
+                            st_v4(dst + 16 * (size_t)u, q[j]);
                         }
+                        if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[j]);
                     }
                 }
             }
         } else {
-            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
+            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - n_tok);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * row_bytes);
                 for (size_t v = tid; v < row_bytes / 16; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
                 zero_scales(a, row, nscales);
             }
         }
+        if (tid < a.K) s_slot[buf ^ 1][tid] = slot_next;
+#pragma unroll
+        for (int j = 0; j < UPT; ++j) {
+            raw[j][0] = nraw[j][0];
+            raw[j][1] = nraw[j][1];
+        }
+        buf ^= 1;
         __syncthreads();
     }
 }
@@ -577,7 +657,7 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             for (int j = 0; j < UPT; ++j) {
                 float f[16];
                 unpack16(raw[j][0], raw[j][1], f);
-                raw[j][0] = quant16<QUANT>(f, sc);
+                raw[j][0] = quant16<QUANT, false>(f, sc);
             }
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[k];

@@ -174,6 +174,51 @@ def test_e4m3_and_int8_conversion_exhaustive_over_bf16(cuda_device):
         assert_rows_equal(cfg, recv_x, recv_scales, ref["recv_x"], ref["recv_scales"])
 
 
+def _groups_over_every_scale(seed):
+    """One 128-channel group per finite positive bf16 group maximum A (all
+    32640 of them, subnormal and huge included): channel 0 holds A, so the
+    group's scale is max(A, 1e-4) / qmax, and channels 1..127 hold x values
+    with |x| <= A -- 64 significands at A's exponent, 32 one binade lower, 24
+    at random lower exponents (down into the fp32 subnormals), zeros, and the
+    smallest bf16 subnormal -- with random signs."""
+    rng = np.random.default_rng(seed)
+    amax = np.arange(1, 0x7f80, dtype=np.uint32)                      # bf16 bit patterns, +0 excluded
+    G = amax.size
+    e = (amax >> 7).astype(np.int64)                                  # exponent field (0: subnormal)
+    xs = np.zeros((G, 127), np.int64)
+    sig = rng.integers(0, 128, (G, 120))
+    expo = np.empty((G, 120), np.int64)
+    expo[:, :64] = e[:, None]
+    expo[:, 64:96] = np.maximum(e[:, None] - 1, 0)
+    expo[:, 96:] = (rng.random((G, 24)) * (e[:, None] + 1)).astype(np.int64)
+    xs[:, :120] = (expo << 7) | sig
+    xs[:, 120:124] = 0
+    xs[:, 124:] = 1                                                   # smallest subnormal
+    xs = np.minimum(xs, amax[:, None].astype(np.int64))               # keep |x| <= A
+    xs |= (rng.random((G, 127)) < 0.5).astype(np.int64) << 15         # signs
+    g = np.concatenate([amax[:, None].astype(np.int64), xs], axis=1).astype(np.uint16)
+    return g                                                          # [G, 128] bf16 bits
+
+
+@pytest.mark.parametrize("quant", ["fp8", "int8"])
+def test_quotients_over_every_group_scale(quant, cuda_device):
+    """Every scale a 128-group can have, each against a spread of x values:
+    codes and scales bit for bit against the oracle's IEEE fp32 division."""
+    g = _groups_over_every_scale(11 if quant == "fp8" else 12)
+    H, R = 1024, 8
+    per = H // 128
+    T = -(-g.shape[0] // per)
+    T = -(-T // R) * R
+    flat = np.zeros((T * per, 128), np.uint16)
+    flat[:g.shape[0]] = g
+    cfg = CONFIGS["tiny"].scaled(num_tokens=T, hidden=H, quant=quant, quant_size=128)
+    wl = make_workload(cfg, 0)
+    wl.x = flat.reshape(T, H)
+    (recv_x, recv_scales, _, _, h), _, _ = gpu_dispatch(cfg, wl, cuda_device)
+    ref = oracle.dispatch(wl.x, wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 1, quant, 128, False)
+    assert_rows_equal(cfg, recv_x, recv_scales, ref["recv_x"], ref["recv_scales"])
+
+
 def test_bad_expert_id_sets_status(cuda_device):
     cfg = CONFIGS["tiny"]
     wl = make_workload(cfg, 0)
