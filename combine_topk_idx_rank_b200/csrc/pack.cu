@@ -33,6 +33,12 @@
 #ifndef EP_PACK_IEEE_DIV
 #define EP_PACK_IEEE_DIV 0     // 1: every quotient x / scale by the IEEE division
 #endif
+#ifndef EP_PACK_GROUP_UPT
+#define EP_PACK_GROUP_UPT 1          // 16-channel units per thread per pass of the group kernel
+#endif
+#ifndef EP_PACK_GROUP_MIN_BLOCKS
+#define EP_PACK_GROUP_MIN_BLOCKS 2   // resident CTAs per SM the group kernel's registers must allow
+#endif
 #ifndef EP_PACK_STORE_HINT
 #define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
 #endif
@@ -485,7 +491,7 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 // destination rows into the other half of s_slot) before the current item is
 // quantised and stored, so its loads are in flight during that work.
 template <int QUANT, int G, int UPT>
-__global__ void __launch_bounds__(256) k_pack_group(PackArgs a) {
+__global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_group(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
     __shared__ int s_slot[2][kMaxTopk];
@@ -702,19 +708,20 @@ cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
 
 template <int QUANT>
 cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
+    constexpr int P = EP_PACK_GROUP_UPT;
     const int U = a.H / 16;
-    const int threads = min(256, round_up32((U + 1) / 2));   // 2 units per thread
+    const int threads = min(512 / P, round_up32((U + P - 1) / P));   // P units per thread
     if constexpr (QUANT == kQuantMxfp4) {
         if (a.quant_size != 32) return cudaErrorInvalidValue;
-        return run(k_pack_group<kQuantMxfp4, 32, 2>, threads, a, st);
+        return run(k_pack_group<kQuantMxfp4, 32, P>, threads, a, st);
     }
     switch (a.quant_size) {
-        case 16: return run(k_pack_group<QUANT, 16, 2>, threads, a, st);
-        case 32: return run(k_pack_group<QUANT, 32, 2>, threads, a, st);
-        case 64: return run(k_pack_group<QUANT, 64, 2>, threads, a, st);
-        case 128: return run(k_pack_group<QUANT, 128, 2>, threads, a, st);
-        case 256: return run(k_pack_group<QUANT, 256, 2>, threads, a, st);
-        case 512: return run(k_pack_group<QUANT, 512, 2>, threads, a, st);
+        case 16: return run(k_pack_group<QUANT, 16, P>, threads, a, st);
+        case 32: return run(k_pack_group<QUANT, 32, P>, threads, a, st);
+        case 64: return run(k_pack_group<QUANT, 64, P>, threads, a, st);
+        case 128: return run(k_pack_group<QUANT, 128, P>, threads, a, st);
+        case 256: return run(k_pack_group<QUANT, 256, P>, threads, a, st);
+        case 512: return run(k_pack_group<QUANT, 512, P>, threads, a, st);
         default: return cudaErrorInvalidValue;
     }
 }
