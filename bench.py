@@ -436,6 +436,8 @@ def run_ours(args):
     else:
         dom, dom_bytes, dom_gbs, dom_ms = "k_combine", ab["combine"] / cfg.num_rounds, combine_gbs, combine_ms / cfg.num_rounds
     clocks = sampler.summary(t_wall0, t_wall1)
+    default_launch = (args.mode == "full" and not args.quant and not args.ue8m0 and not args.combine_quant
+                      and not args.tokens)
     # routing (1 cooperative kernel) unless cached, pack x rounds, combine x rounds
     launches_per_step = (0 if args.mode == "cached" else 1) + 2 * cfg.num_rounds
 
@@ -464,7 +466,8 @@ def run_ours(args):
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak, "unit": "GB/s",
                      "peak_kind": peak_kind, "frac": round(dom_gbs / peak, 4),
                      "algorithmic_bytes_per_launch": int(dom_bytes), "launch_ms": round(dom_ms, 5),
-                     "traffic": traffic_for(dom, args.workload)},
+                     # the capture holds the workload's default launch only
+                     "traffic": traffic_for(dom, args.workload) if default_launch else None},
         "e2e": {"value": round(job_tokens_per_s(world, T, e2e_ms / e2e_steps), 1), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms / e2e_steps, 4)},
