@@ -311,13 +311,9 @@ def run_ours(args):
                            num_rounds=cfg.num_rounds, buffers=bufs, events=evs, handle=bufs.handle,
                            scale_ue8m0=ue8)
         elif ll:
-            if evs is not None:
-                evs[0].record()
             ep.ep_dispatch_low_latency(x, ti, tw, M, E, R, q, quant_size=cfg.quant_size,
                                        round_scale=cfg.round_scale, workspace=bufs.workspace, buffers=ll_bufs,
-                                       scale_ue8m0=ue8)
-            if evs is not None:
-                evs[1].record()
+                                       scale_ue8m0=ue8, events=evs)
         else:
             ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
                            quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,

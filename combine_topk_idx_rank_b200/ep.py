@@ -402,13 +402,14 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
                             quant: Optional[str] = None, *, quant_size: int = 128, round_scale: bool = False,
                             workspace: Optional[torch.Tensor] = None, buffers: Optional[dict] = None,
                             cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
-                            scale_ue8m0: bool = False):
+                            scale_ue8m0: bool = False, events: Optional[tuple] = None):
     """Low-latency (decode) dispatch into fixed-capacity per-expert buffers.
 
     Returns (recv_x [E, R*M, H], recv_scales [E, R*M, H/quant_size] or None,
     packed_recv_count [E], packed_recv_layout_range [E, R] int64, handle);
     entry (t,k) of source rank r for expert e is row r*M + p of expert e's
-    block, p its position among rank r's entries for e.
+    block, p its position among rank r's entries for e.  ``events`` (two
+    recorded torch.cuda.Event) bracket the pack kernel, as in ep_dispatch.
     """
     _need_cuda(x, "x", torch.bfloat16)
     _need_cuda(topk_idx, "topk_idx", torch.int64)
@@ -437,7 +438,9 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
         workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
     opts = _Opts(1, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), 1, int(bool(scale_ue8m0)),
                  None if cumulative_local_expert_recv_stats is None
-                 else cumulative_local_expert_recv_stats.data_ptr(), None, None)
+                 else cumulative_local_expert_recv_stats.data_ptr(),
+                 None if events is None else events[0].cuda_event,
+                 None if events is None else events[1].cuda_event)
     ch = h._c()
     st = _lib.ep_dispatch_low_latency(_ptr(x), T, H, _ptr(topk_idx), _ptr(topk_weights), K, E, R, M, C.byref(opts),
                                       _ptr(b["recv_x"]), _ptr(b["recv_scales"]), _ptr(b["recv_topk_idx"]),

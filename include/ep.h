@@ -186,9 +186,10 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
  *   handle               as in ep_dispatch (recv_src_metadata has E*R*M rows);
  *                        low_latency = 1, recv_capacity = E*R*M; psum holds the
  *                        inclusive prefix of the unaligned counts
- * opts->expert_alignment must be 1.  More than M entries of one (expert, rank)
- * set EP_ERR_CAPACITY (they are dropped).  ep_combine and ep_dispatch_cached
- * accept the handle.
+ * opts->expert_alignment must be 1; opts->num_rounds must divide T/R; the
+ * optional pack events bracket the pack kernel as in ep_dispatch.  More than M
+ * entries of one (expert, rank) set EP_ERR_CAPACITY (they are dropped).
+ * ep_combine and ep_dispatch_cached accept the handle.
  */
 ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
                                     const float* topk_weights, int32_t K, int32_t E, int32_t R,
