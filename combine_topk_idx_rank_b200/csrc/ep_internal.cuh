@@ -105,7 +105,8 @@ struct RouteArgs {
 struct PackArgs {
     const uint16_t* x;
     int H, K, E;
-    const int32_t* dst_slot;    // [T,K] received row of each entry (-1 = none)
+    const int32_t* dst_slot;    // [T,K] received row of each entry (-1 = none); a row at or
+                                // past capacity is skipped and reported as EP_ERR_CAPACITY
     uint8_t* recv_x;
     float* recv_scales;
     int64_t capacity;

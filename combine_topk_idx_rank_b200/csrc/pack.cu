@@ -386,7 +386,9 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
             fence_proxy_async_smem();
             for (int k = 0; k < K; ++k) {
                 const int slot = sslot[s * kMaxTopk + k];
-                if (slot >= 0) bulk_store(a.recv_x + (int64_t)slot * row_bytes + off, stage + (size_t)s * chunk_bytes, bytes);
+                if (slot >= a.capacity) set_error(a.err, EP_ERR_CAPACITY);
+                else if (slot >= 0)
+                    bulk_store(a.recv_x + (int64_t)slot * row_bytes + off, stage + (size_t)s * chunk_bytes, bytes);
             }
             bulk_commit();
             bulk_wait_read<1>();   // the stores of unit i-1 have read their stage
@@ -463,6 +465,10 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
                 for (int k = 0; k < a.K; ++k) {
                     const int slot = s_slot[k];
                     if (slot < 0) continue;
+                    if (slot >= a.capacity) {
+                        set_error(a.err, EP_ERR_CAPACITY);
+                        continue;
+                    }
                     uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)slot * a.H * 2);
 #pragma unroll
                     for (int u = 0; u < VPT; ++u) {
@@ -574,6 +580,10 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[buf][k];
                 if (slot < 0) continue;
+                if (slot >= a.capacity) {
+                    set_error(a.err, EP_ERR_CAPACITY);
+                    continue;
+                }
                 uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
@@ -668,6 +678,10 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[k];
                 if (slot < 0) continue;
+                if (slot >= a.capacity) {
+                    set_error(a.err, EP_ERR_CAPACITY);
+                    continue;
+                }
                 uint8_t* dst = a.recv_x + (size_t)slot * a.H;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {

@@ -7,6 +7,8 @@ hidden, duplicate ids, group sizes 16..512, per-token FP8, power-of-two int8
 scales).  Bit-exact for layout, slots, metadata, rows, codes and scales;
 combine is bit-exact too and also meets the 1e-2 relative contract.
 """
+import copy
+
 import numpy as np
 import pytest
 import torch
@@ -16,7 +18,7 @@ from combine_topk_idx_rank_b200 import ep
 from combine_topk_idx_rank_b200.workloads import CONFIGS, make_workload, make_y
 
 from gpu_parity import (assert_combine_close, assert_layout_equal, assert_rows_equal, assert_slots_equal,
-                        gpu_dispatch, to_dev, u16)
+                        gpu_dispatch, to_dev, u8, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -305,6 +307,45 @@ def test_cached_dispatch_repacks_new_rows(name, cuda_device):
     ref_x, ref_s = oracle.dispatch_rows(wl2.x, slots["dst_buffer_slot_idx"], cfg.quant, cfg.quant_size,
                                         cfg.round_scale, num_rows=rows)
     assert_rows_equal(cfg, rx, rs, ref_x, ref_s)
+
+
+@pytest.mark.parametrize("quant,qs", [(None, 128), ("fp8", 128), ("int8", 512)])
+def test_pack_skips_and_reports_rows_past_capacity(quant, qs, cuda_device):
+    """The pack kernels write no row at or past recv_capacity, whatever the
+    handle's dst_buffer_slot_idx holds: such entries are skipped and reported
+    as EP_ERR_CAPACITY, the others are packed as usual (bulk bf16, group and
+    per-token quantisation)."""
+    cfg = CONFIGS["tiny"].scaled(hidden=512)
+    wl = make_workload(cfg, 4)
+    x, ti, tw = to_dev(wl, cuda_device)
+    (_, _, _, _, h), _, _ = gpu_dispatch(cfg, wl, cuda_device)
+    need = h.num_recv_rows
+    full = ep.alloc_dispatch_buffers(cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks,
+                                     1, quant, qs, recv_capacity=need + 64, device=cuda_device)
+    full.recv_x.view(torch.uint8).fill_(0x5A)
+    cut = need - 8                           # rows cut..need-1 now lie past the capacity
+    h2 = copy.copy(h)
+    h2.recv_capacity = cut
+    h2.err = torch.zeros_like(h.err)
+    slots = h.dst_buffer_slot_idx.clone()
+    slots[5, 0] = cut + 40                   # and a few more, inside the guard rows
+    slots[9, 1] = cut + 63
+    h2.dst_buffer_slot_idx = slots
+    rs = None if full.recv_scales is None else full.recv_scales[:cut]
+    short = ep.DispatchBuffers(full.recv_x[:cut], rs, full.recv_topk_idx, full.recv_topk_weights, h2,
+                               full.workspace, quant, qs)
+    ep.ep_dispatch(x, quant=quant, quant_size=qs, buffers=short, handle=h2)
+    torch.cuda.synchronize()
+    assert h2.read_error() == ep.EP_ERR_CAPACITY
+    assert torch.all(full.recv_x[cut:].contiguous().view(torch.uint8) == 0x5A)
+    dst = slots.cpu().numpy()
+    ref_x, ref_s = oracle.dispatch_rows(wl.x, np.where(dst < cut, dst, -1), quant or "none", qs, False,
+                                        num_rows=cut)
+    got = u16(full.recv_x[:cut]) if quant is None else u8(full.recv_x[:cut]).reshape(cut, -1)
+    written = np.unique(dst[(dst >= 0) & (dst < cut)])
+    assert np.array_equal(got[written], ref_x[written])
+    if quant is not None:
+        assert np.array_equal(rs.cpu().numpy()[written].view(np.uint32), ref_s[written].view(np.uint32))
 
 
 def test_cached_dispatch_rejects_routing_args(cuda_device):
