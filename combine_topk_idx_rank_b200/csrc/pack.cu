@@ -1,13 +1,16 @@
 // Permute / pack: every source token's row is read from HBM once and written
 // to each of its received rows (one per unmasked top-k entry, rows already
-// resolved by k_slots into dst_buffer_slot_idx), as a bf16 bit copy or
+// resolved by k_route into dst_buffer_slot_idx), as a bf16 bit copy or
 // quantised once per token on the fly:
 //   - FP8 e4m3 (OCP e4m3fn) or int8 with one fp32 scale per quant_size
 //     channels: scale = max(amax, 1e-4) / 448 (or / 127) by IEEE division,
 //     optionally rounded up to a power of two (round_scale / use_ue8m0 of
-//     low_latency_dispatch, "DeepEP communication library guide v2.1"),
-//     codes = RNE-saturating conversion of x / scale (IEEE division);
-//   - quant_size = 128 (group) or hidden (per token) (guide v2.1, 1.3.1).
+//     low_latency_dispatch, "DeepEP communication library guide v2.1") and
+//     then optionally stored as its UE8M0 byte; codes = RNE-saturating
+//     conversion of the IEEE quotient x / scale;
+//   - MXFP4 (use_mxfp4, groups of 32): E2M1 codes of x / 2^(floor(log2 amax) - 2)
+//     with the scale stored as its UE8M0 byte (the OCP MX conversion);
+//   - quant_size = 16..512 (group) or hidden (per token) (guide v2.1, 1.3.1).
 // The same persistent grid zero-fills the padding rows that expert alignment
 // adds (comparative analysis, section 3.1).
 //
