@@ -53,6 +53,9 @@ __device__ bool grid_barrier(unsigned* counter, unsigned target, int* s_flag) {
     return *s_flag != 0;
 }
 
+// Rank of expert e (e / L): a shift when L is a power of two (sh >= 0).
+__device__ __forceinline__ int rank_of(int e, int L, int sh) { return sh >= 0 ? e >> sh : e / L; }
+
 // Inclusive scan of one value per thread over the block (blockDim.x = 256).
 __device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -127,6 +130,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
+    const int shL = (L & (L - 1)) == 0 ? __ffs(L) - 1 : -1;
     const unsigned lt = lanemask_lt();
     const int per_warp = ((C * K / kRouteWarps) + 31) & ~31;   // entries per warp, a multiple of 32
     const int nb = per_warp / 32;
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         for (int tl = tid; tl < nt; tl += kRouteThreads) {
             for (int k = 0; k < K; ++k) {
                 const int e = s_idx[tl * K + k];
-                if (e >= 0) s_inr[tl * R + e / L] = 1;
+                if (e >= 0) s_inr[tl * R + rank_of(e, L, shL)] = 1;
             }
         }
         __syncthreads();
@@ -346,7 +350,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             a.dst_slot[e0 + i] = slot;
             if (slot < 0) continue;
             reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t0 + tl, k);
-            const int rdst = e / L;
+            const int rdst = rank_of(e, L, shL);
+            const int lo = rdst * L;   // local ids of the receiving rank: [lo, lo + L)
             const int* ids = s_idx + tl * K;
             const float* ws = s_w + tl * K;
             if constexpr (KT > 0) {
@@ -359,8 +364,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int ej = ids[j + u];
-                        const bool here = ej >= 0 && ej / L == rdst;
-                        o[u] = here ? ej - rdst * L : -1;
+                        const bool here = (unsigned)(ej - lo) < (unsigned)L;
+                        o[u] = here ? ej - lo : -1;
                         w[u] = here ? ws[j + u] : 0.0f;
                     }
                     ri[j / 4] = make_int4(o[0], o[1], o[2], o[3]);
@@ -371,8 +376,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
                 float* rw = a.recv_topk_weights + (int64_t)slot * K;
                 for (int j = 0; j < K; ++j) {
                     const int ej = ids[j];
-                    const bool here = ej >= 0 && ej / L == rdst;
-                    ri[j] = here ? ej - rdst * L : -1;
+                    const bool here = (unsigned)(ej - lo) < (unsigned)L;
+                    ri[j] = here ? ej - lo : -1;
                     rw[j] = here ? ws[j] : 0.0f;
                 }
             }
