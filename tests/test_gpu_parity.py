@@ -103,6 +103,15 @@ def test_quant_variants(quant, qs, rs, cuda_device):
     run_and_compare(cfg, 0, cuda_device)
 
 
+@pytest.mark.parametrize("quant,H", [("int8", 16384), ("fp8", 24576), ("int8", 65536)])
+def test_per_token_quant_large_hidden(quant, H, cuda_device):
+    """Per-token quantisation of long rows: up to 1024 units of 16 channels
+    run two units per thread in blocks of up to 512, up to 2048 in blocks of
+    1024, longer rows four units per thread."""
+    cfg = CONFIGS["decode"].scaled(num_tokens=16 * 3, hidden=H, quant=quant, quant_size=H, expert_alignment=4)
+    run_and_compare(cfg, 0, cuda_device)
+
+
 def test_edge_shapes(cuda_device):
     base = CONFIGS["tiny"]
     cases = [
