@@ -307,7 +307,7 @@ __device__ __forceinline__ float finish_scale(float amax, float qmax, int round_
 }
 
 // Loads the K received rows of token t into s_slot (threads 0..K-1).
-__device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
+[[maybe_unused]] __device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
     if (threadIdx.x < a.K) s_slot[threadIdx.x] = a.dst_slot[(int64_t)t * a.K + threadIdx.x];
 }
 
