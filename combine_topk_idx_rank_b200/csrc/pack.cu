@@ -306,9 +306,20 @@ __device__ __forceinline__ float finish_scale(float amax, float qmax, int round_
     return round_scale ? pow2_ceil_bits(s) : s;
 }
 
+// A destination row as the pack kernels use it: rows at or past the receive
+// capacity (a handle with foreign rows, or slots left stale by routing that
+// stopped on an error) are reported as EP_ERR_CAPACITY and dropped (-1).
+__device__ __forceinline__ int checked_row(const PackArgs& a, int slot) {
+    if (slot >= a.capacity) {
+        set_error(a.err, EP_ERR_CAPACITY);
+        return -1;
+    }
+    return slot;
+}
+
 // Loads the K received rows of token t into s_slot (threads 0..K-1).
 [[maybe_unused]] __device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
-    if (threadIdx.x < a.K) s_slot[threadIdx.x] = a.dst_slot[(int64_t)t * a.K + threadIdx.x];
+    if (threadIdx.x < a.K) s_slot[threadIdx.x] = checked_row(a, a.dst_slot[(int64_t)t * a.K + threadIdx.x]);
 }
 
 }  // namespace
@@ -363,7 +374,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         int t, c;
         unit(j, t, c);
         if (lane == 0) issue_load(j, t, c);
-        if (lane < K) sslot[(j % S) * kMaxTopk + lane] = a.dst_slot[(int64_t)t * K + lane];
+        if (lane < K) sslot[(j % S) * kMaxTopk + lane] = checked_row(a, a.dst_slot[(int64_t)t * K + lane]);
     }
     __syncwarp();
 
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
     for (; i < n_mine; ++i) {
         const int s = i % S;
         // slots fetched last iteration belong to unit i + S - 2
-        if (i >= 1 && i + S - 2 < n_mine && lane < K) sslot[((i + S - 2) % S) * kMaxTopk + lane] = pending;
+        if (i >= 1 && i + S - 2 < n_mine && lane < K) sslot[((i + S - 2) % S) * kMaxTopk + lane] = checked_row(a, pending);
         // lane 0 waits for the stage; the verdict is broadcast so the warp stays converged
         int landed = lane == 0 ? (int)mbar_wait(&mbar[s], (uint32_t)((i / S) & 1)) : 0;
         landed = __shfl_sync(0xffffffffu, landed, 0);
@@ -389,8 +400,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
             fence_proxy_async_smem();
             for (int k = 0; k < K; ++k) {
                 const int slot = sslot[s * kMaxTopk + k];
-                if (slot >= a.capacity) set_error(a.err, EP_ERR_CAPACITY);
-                else if (slot >= 0)
+                if (slot >= 0)
                     bulk_store(a.recv_x + (int64_t)slot * row_bytes + off, stage + (size_t)s * chunk_bytes, bytes);
             }
             bulk_commit();
@@ -468,10 +478,6 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
                 for (int k = 0; k < a.K; ++k) {
                     const int slot = s_slot[k];
                     if (slot < 0) continue;
-                    if (slot >= a.capacity) {
-                        set_error(a.err, EP_ERR_CAPACITY);
-                        continue;
-                    }
                     uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)slot * a.H * 2);
 #pragma unroll
                     for (int u = 0; u < VPT; ++u) {
@@ -546,7 +552,7 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
     int slot_next = -1;
     int item = blockIdx.x;
     if (item < n_tok) fetch(item, raw, slot_next);
-    if (tid < a.K) s_slot[0][tid] = slot_next;
+    if (tid < a.K) s_slot[0][tid] = checked_row(a, slot_next);
     __syncthreads();
     int buf = 0;
     for (; item < n_items; item += gridDim.x) {
@@ -583,10 +589,6 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[buf][k];
                 if (slot < 0) continue;
-                if (slot >= a.capacity) {
-                    set_error(a.err, EP_ERR_CAPACITY);
-                    continue;
-                }
                 uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
@@ -609,7 +611,7 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
                 zero_scales(a, row, nscales);
             }
         }
-        if (tid < a.K) s_slot[buf ^ 1][tid] = slot_next;
+        if (tid < a.K) s_slot[buf ^ 1][tid] = checked_row(a, slot_next);
 #pragma unroll
         for (int j = 0; j < UPT; ++j) {
             raw[j][0] = nraw[j][0];
@@ -661,7 +663,7 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
     int slot_next = -1;
     int item = blockIdx.x;
     if (item < n_tok) fetch(item, raw, slot_next);
-    if (tid < a.K) s_slot[0][tid] = slot_next;
+    if (tid < a.K) s_slot[0][tid] = checked_row(a, slot_next);
     __syncthreads();
     int buf = 0;
     // with 4 units per thread (rows above 32768 channels) the next row is
@@ -710,10 +712,6 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[buf][k];
                 if (slot < 0) continue;
-                if (slot >= a.capacity) {
-                    set_error(a.err, EP_ERR_CAPACITY);
-                    continue;
-                }
                 uint8_t* dst = a.recv_x + (size_t)slot * a.H;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
@@ -739,7 +737,7 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
         } else {
             if (nxt < n_tok) fetch(nxt, raw, slot_next);
         }
-        if (tid < a.K) s_slot[buf ^ 1][tid] = slot_next;
+        if (tid < a.K) s_slot[buf ^ 1][tid] = checked_row(a, slot_next);
         buf ^= 1;
         __syncthreads();
     }
