@@ -318,7 +318,7 @@ __device__ __forceinline__ int checked_row(const PackArgs& a, int slot) {
 }
 
 // Loads the K received rows of token t into s_slot (threads 0..K-1).
-[[maybe_unused]] __device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
+__device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot) {
     if (threadIdx.x < a.K) s_slot[threadIdx.x] = checked_row(a, a.dst_slot[(int64_t)t * a.K + threadIdx.x]);
 }
 
@@ -624,14 +624,12 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
 
 // ----------------------------------------------- per-token quantisation (G=H)
 // The whole row stays in registers (UPT units of 16 channels per thread) while
-// the block reduces its amax.  As in the group kernel, the CTA's next token
-// row and its destination rows are fetched before the current row is reduced,
-// quantised and stored.  MAXT bounds the block (and so the registers).
-template <int QUANT, int UPT, int MAXT>
-__global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
+// the block reduces its amax.
+template <int QUANT, int UPT>
+__global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
-    __shared__ int s_slot[2][kMaxTopk];
+    __shared__ int s_slot[kMaxTopk];
     __shared__ float s_red[33];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
@@ -639,50 +637,23 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
     const int nwarps = blockDim.x >> 5;
     const int U = a.H / 16;
     const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
-    const int n_tok = a.n_tok_items;
-    const int n_items = n_tok + n_pad;
-
-    // issues the loads of token item `item`: its units into r, its rows into slot
-    auto fetch = [&](int item, uint4 (&r)[UPT][2], int& slot) {
-        const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
-        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
+    const int n_items = a.n_tok_items + n_pad;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        if (item < a.n_tok_items) {
+            const int t = token_of_item(item, a.tokens_per_rank, a.per_round, a.round);
+            load_slots(a, t, s_slot);
+            const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
+            uint4 raw[UPT][2];
 #pragma unroll
-        for (int j = 0; j < UPT; ++j) {
-            const int u = j * blockDim.x + tid;
-            if (u < U) {
-                r[j][0] = ld_nc_v4(xr + 2 * u);
-                r[j][1] = ld_nc_v4(xr + 2 * u + 1);
-            } else {
-                r[j][0] = r[j][1] = make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < UPT; ++j) {
+                const int u = j * blockDim.x + tid;
+                if (u < U) {
+                    raw[j][0] = ld_nc_v4(xr + 2 * u);
+                    raw[j][1] = ld_nc_v4(xr + 2 * u + 1);
+                } else {
+                    raw[j][0] = raw[j][1] = make_uint4(0, 0, 0, 0);
+                }
             }
-        }
-        slot = tid < a.K ? a.dst_slot[(int64_t)t * a.K + tid] : -1;
-    };
-
-    uint4 raw[UPT][2];
-    int slot_next = -1;
-    int item = blockIdx.x;
-    if (item < n_tok) fetch(item, raw, slot_next);
-    if (tid < a.K) s_slot[0][tid] = checked_row(a, slot_next);
-    __syncthreads();
-    int buf = 0;
-    // with 4 units per thread (rows above 32768 channels) the next row is
-    // fetched after the current one is stored instead: two rows of registers
-    // would spill
-    constexpr bool kAhead = UPT <= 2;
-    for (; item < n_items; item += gridDim.x) {
-        const int nxt = item + gridDim.x;
-        uint4 nraw[kAhead ? UPT : 1][2];
-        slot_next = -1;
-        if constexpr (kAhead) {
-            if (nxt < n_tok) {
-                fetch(nxt, nraw, slot_next);
-            } else {
-#pragma unroll
-                for (int j = 0; j < UPT; ++j) nraw[j][0] = nraw[j][1] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        if (item < n_tok) {
             float m = 0.0f;
 #pragma unroll
             for (int j = 0; j < UPT; ++j) {
@@ -710,7 +681,7 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
                 raw[j][0] = quant16<QUANT, false>(f, sc);
             }
             for (int k = 0; k < a.K; ++k) {
-                const int slot = s_slot[buf][k];
+                const int slot = s_slot[k];
                 if (slot < 0) continue;
                 uint8_t* dst = a.recv_x + (size_t)slot * a.H;
 #pragma unroll
@@ -721,24 +692,13 @@ __global__ void __launch_bounds__(MAXT) k_pack_token(PackArgs a) {
                 if (tid == 0) store_scale(a, (size_t)slot, sc);
             }
         } else {
-            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - n_tok);
+            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
             if (row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
                 if (tid == 0) zero_scales(a, row, 1);
             }
         }
-        if constexpr (kAhead) {
-#pragma unroll
-            for (int j = 0; j < UPT; ++j) {
-                raw[j][0] = nraw[j][0];
-                raw[j][1] = nraw[j][1];
-            }
-        } else {
-            if (nxt < n_tok) fetch(nxt, raw, slot_next);
-        }
-        if (tid < a.K) s_slot[buf ^ 1][tid] = checked_row(a, slot_next);
-        buf ^= 1;
         __syncthreads();
     }
 }
@@ -784,9 +744,12 @@ cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
 template <int QUANT>
 cudaError_t launch_token(const PackArgs& a, cudaStream_t st) {
     const int U = a.H / 16;
-    if (U <= 1024) return run(k_pack_token<QUANT, 2, 512>, round_up32((U + 1) / 2), a, st);
-    if (U <= 2 * 1024) return run(k_pack_token<QUANT, 2, 1024>, round_up32((U + 1) / 2), a, st);
-    return run(k_pack_token<QUANT, 4, 1024>, min(1024, round_up32((U + 3) / 4)), a, st);
+    if (U <= 2 * 1024) {
+        const int threads = min(1024, round_up32((U + 1) / 2));
+        return run(k_pack_token<QUANT, 2>, threads, a, st);
+    }
+    const int threads = min(1024, round_up32((U + 3) / 4));
+    return run(k_pack_token<QUANT, 4>, threads, a, st);
 }
 
 cudaError_t launch_bulk(const PackArgs& a, cudaStream_t st) {
