@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import ctypes as C
 import dataclasses
+import functools
 import os
 from typing import List, Optional
 
@@ -119,6 +120,19 @@ def workspace_bytes(T: int, K: int, E: int, R: int) -> int:
     return int(_lib.ep_workspace_bytes(T, K, E, R))
 
 
+def _on_tensor_device(fn):
+    """Runs a call with its first argument's GPU as the current device, so that
+    the library launches on the device whose stream it is given."""
+    @functools.wraps(fn)
+    def call(*args, **kw):
+        t = args[0] if args else None
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            with torch.cuda.device(t.device):
+                return fn(*args, **kw)
+        return fn(*args, **kw)
+    return call
+
+
 def _need_cuda(t: torch.Tensor, name: str, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -165,7 +179,8 @@ class EPHandle:
 
     def read_error(self) -> int:
         st = C.c_int32(0)
-        _check(_lib.ep_read_error(_ptr(self.err), _stream(self.err.device), C.byref(st)), "ep_read_error")
+        with torch.cuda.device(self.err.device):
+            _check(_lib.ep_read_error(_ptr(self.err), _stream(self.err.device), C.byref(st)), "ep_read_error")
         return st.value
 
     def check(self):
@@ -226,6 +241,7 @@ def alloc_dispatch_buffers(num_tokens: int, hidden: int, num_topk: int, num_expe
                            q, quant_size)
 
 
+@_on_tensor_device
 def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int,
                            workspace: Optional[torch.Tensor] = None, check: bool = True):
     """Routing histogram: (num_tokens_per_rank [R] i32, num_tokens_per_expert [E] i32,
@@ -278,6 +294,7 @@ def _dispatch_cached(x, handle: EPHandle, quant, quant_size, round_scale, num_ro
     return recv_x, recv_scales, None, None, h
 
 
+@_on_tensor_device
 def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
                 topk_weights: Optional[torch.Tensor] = None, expert_alignment: int = 1,
                 quant: Optional[str] = None, *, num_experts: Optional[int] = None,
@@ -352,6 +369,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
     return recv_x, recv_scales, rti, rtw, h
 
 
+@_on_tensor_device
 def ep_combine(y: torch.Tensor, handle: EPHandle, topk_weights: torch.Tensor,
                out: Optional[torch.Tensor] = None, *, y_scales: Optional[torch.Tensor] = None,
                quant_size: int = 128, shared: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -397,6 +415,7 @@ def ep_combine(y: torch.Tensor, handle: EPHandle, topk_weights: torch.Tensor,
     return out
 
 
+@_on_tensor_device
 def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
                             num_max_dispatch_tokens_per_rank: int, num_experts: int, num_ranks: int,
                             quant: Optional[str] = None, *, quant_size: int = 128, round_scale: bool = False,
