@@ -98,13 +98,16 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
 }
 
 // Quantisation options shared by ep_dispatch and ep_dispatch_cached.
-bool quant_ok(int quant, int quant_size, int H, const float* recv_scales) {
+// The quantisation is a supported one for rows of H channels; the scales
+// array is required as soon as there is a row to hold (rows > 0).
+bool quant_ok(int quant, int quant_size, int H, const float* recv_scales, int64_t rows) {
     if (quant == EP_QUANT_NONE) return true;
-    if (quant == EP_QUANT_MXFP4) return quant_size == 32 && H % 32 == 0 && recv_scales != nullptr;
+    const bool scales = recv_scales != nullptr || rows == 0;
+    if (quant == EP_QUANT_MXFP4) return quant_size == 32 && H % 32 == 0 && scales;
     if (quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8) return false;
     const bool group = quant_size == 16 || quant_size == 32 || quant_size == 64 || quant_size == 128 ||
                        quant_size == 256 || quant_size == 512;
-    return H % 16 == 0 && (quant_size == H || group) && H % quant_size == 0 && recv_scales != nullptr;
+    return H % 16 == 0 && (quant_size == H || group) && H % quant_size == 0 && scales;
 }
 
 }  // namespace
@@ -169,7 +172,7 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     if (ep_recv_capacity_bound(T, K, E, A) >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
     if (recv_capacity < 0 || recv_capacity >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
-    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (!quant_ok(quant, quant_size, H, recv_scales, recv_capacity)) return EP_ERR_INVALID_ARG;
     if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
         return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
@@ -229,7 +232,7 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
     if (rows >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
     const int quant = opts->quant;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
-    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (!quant_ok(quant, quant_size, H, recv_scales, rows)) return EP_ERR_INVALID_ARG;
     if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
         return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
@@ -279,7 +282,7 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
     if (H < 8 || H > 65536 || H % 8 != 0 || rounds < 1 || (T / R) % rounds != 0) return EP_ERR_INVALID_ARG;
     const int quant = opts->quant;
     const int quant_size = quant == EP_QUANT_NONE ? 0 : opts->quant_size;
-    if (!quant_ok(quant, quant_size, H, recv_scales)) return EP_ERR_INVALID_ARG;
+    if (!quant_ok(quant, quant_size, H, recv_scales, h->recv_capacity)) return EP_ERR_INVALID_ARG;
     if (opts->scale_ue8m0 && (quant == EP_QUANT_FP8_E4M3 || quant == EP_QUANT_INT8) && !opts->round_scale)
         return EP_ERR_INVALID_ARG;   // UE8M0 bytes hold powers of two only
     if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
@@ -303,7 +306,8 @@ ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant,
     if (h->err == nullptr) return EP_ERR_INVALID_ARG;
     if (y_quant == EP_QUANT_MXFP4) return EP_ERR_INVALID_ARG;   // combine reads FP8 / int8 codes only
     const int qs = y_quant == EP_QUANT_NONE ? 0 : y_quant_size;
-    if (!quant_ok(y_quant, qs, H, y_quant == EP_QUANT_NONE ? nullptr : y_scales)) return EP_ERR_INVALID_ARG;
+    if (!quant_ok(y_quant, qs, H, y_quant == EP_QUANT_NONE ? nullptr : y_scales, h->recv_capacity))
+        return EP_ERR_INVALID_ARG;
     if (T > 0 && (out == nullptr || topk_weights == nullptr || h->dst_buffer_slot_idx == nullptr))
         return EP_ERR_INVALID_ARG;
     if (h->recv_capacity > 0 && y == nullptr) return EP_ERR_INVALID_ARG;

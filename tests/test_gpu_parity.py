@@ -130,8 +130,11 @@ def test_edge_shapes(cuda_device):
         run_and_compare(cfg, 0, cuda_device)
 
 
-def test_no_tokens(cuda_device):
-    cfg = CONFIGS["prefill"].scaled(num_tokens=0, hidden=256)
+@pytest.mark.parametrize("quant,qs", [("none", 128), ("fp8", 128), ("mxfp4", 32)])
+def test_no_tokens(quant, qs, cuda_device):
+    # with no tokens and alignment 1 the receive capacity is zero: empty outputs, no scales array needed
+    cfg = CONFIGS["prefill"].scaled(num_tokens=0, hidden=256, quant=quant, quant_size=qs,
+                                    expert_alignment=1 if quant != "none" else 128)
     wl = make_workload(cfg, 0)
     (recv_x, _, rti, rtw, h), lay, _ = gpu_dispatch(cfg, wl, cuda_device)
     assert h.num_recv_rows == 0
