@@ -19,7 +19,7 @@ from gpu_parity import assert_layout_equal, assert_slots_equal, to_dev, u8, u16
 
 pytestmark = pytest.mark.gpu
 
-N_CASES = 48
+N_CASES = 96
 
 
 def _draw(i):
@@ -118,3 +118,46 @@ def test_random_configuration_low_latency(i, cuda_device):
     if q is not None:
         gs = recv_s.reshape(rows, -1).cpu().numpy()
         assert np.array_equal(gs[used].view(np.uint32), ref_s[used].view(np.uint32))
+
+
+@pytest.mark.parametrize("i", range(1, N_CASES, 2))
+def test_random_cached_dispatch_and_quantised_combine(i, cuda_device):
+    """On the same draws: the layout call alone; a cached dispatch of new
+    activations with the first call's routing; and, for FP8 / int8 codes with
+    fp32 scales, the combine of the received codes with a shared-expert row."""
+    dev = cuda_device
+    cfg, ue8 = _draw(i)
+    T, H, K, E, R, A = (cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks,
+                        cfg.expert_alignment)
+    q = None if cfg.quant == "none" else cfg.quant
+    wl = make_workload(cfg, seed=i)
+    x, ti, tw = to_dev(wl, dev)
+    assert_layout_equal(ep.ep_get_dispatch_layout(ti, E, R), oracle.layout(wl.topk_idx, E, R))
+    bufs = ep.alloc_dispatch_buffers(T, H, K, E, R, A, q, cfg.quant_size, cfg.num_rounds, device=dev,
+                                     scale_ue8m0=ue8)
+    kw = dict(quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds, buffers=bufs,
+              scale_ue8m0=ue8)
+    ep.ep_dispatch(x, ti, tw, A, q, num_experts=E, num_ranks=R, **kw)
+    s = oracle.slots(wl.topk_idx, wl.topk_weights, E, R, A)
+    n = s["num_recv_rows"]
+    wl2 = make_workload(cfg, seed=i + 500)
+    x2 = torch.from_numpy(wl2.x.view(np.int16)).view(torch.bfloat16).to(dev)
+    rx, rs, _, _, _ = ep.ep_dispatch(x2, quant=q, handle=bufs.handle, **kw)
+    torch.cuda.synchronize()
+    bufs.handle.check()
+    if n == 0:
+        return
+    ref_x, ref_s = oracle.dispatch_rows_mx(wl2.x, s["dst_buffer_slot_idx"], cfg.quant, cfg.quant_size,
+                                           cfg.round_scale, ue8, num_rows=n)
+    got = u16(rx).view(np.uint8).reshape(n, -1) if q is None else u8(rx).reshape(n, -1)
+    assert np.array_equal(got, ref_x.reshape(n, -1))
+    if q in ("fp8", "int8") and not ue8:
+        shared_np = make_y(T, H, i + 7)
+        shared = torch.from_numpy(shared_np.view(np.int16)).view(torch.bfloat16).to(dev)
+        out = ep.ep_combine(bufs.recv_x, bufs.handle, tw, y_scales=bufs.recv_scales, quant_size=cfg.quant_size,
+                            shared=shared)
+        torch.cuda.synchronize()
+        bufs.handle.check()
+        ref_out = oracle.combine_rows_q(ref_x.reshape(n, -1), ref_s, cfg.quant, cfg.quant_size,
+                                        s["dst_buffer_slot_idx"], wl.topk_weights, shared_np)
+        assert np.array_equal(u16(out), ref_out)
