@@ -142,6 +142,25 @@ def test_no_tokens(quant, qs, cuda_device):
     assert torch.all(lay[0] == 0) and torch.all(lay[1] == 0)
 
 
+def test_more_chunks_than_resident_ctas(cuda_device):
+    """8 ranks x 16384 tokens: 512 routing chunks of 256 tokens, more than the
+    cooperative grid holds at once (3 CTAs per SM), so each CTA routes several
+    chunks and phase 3 reloads their ids and ranks from global memory; normal
+    and low-latency layouts, hidden 64 to keep the rows small."""
+    cfg = CONFIGS["prefill"].scaled(num_tokens=8 * 16384, hidden=64, expert_alignment=16)
+    wl, _, _ = run_and_compare(cfg, 6, cuda_device)
+    x, ti, tw = to_dev(wl, cuda_device)
+    T, E, R = cfg.num_tokens, cfg.num_experts, cfg.num_ranks
+    M = T // R
+    _, _, count, layout_range, h = ep.ep_dispatch_low_latency(x, ti, tw, M, E, R)
+    torch.cuda.synchronize()
+    h.check()
+    ref = oracle.ll_slots(wl.topk_idx, wl.topk_weights, E, R, M)
+    assert np.array_equal(h.dst_buffer_slot_idx.cpu().numpy(), ref["dst_buffer_slot_idx"])
+    assert np.array_equal(count.cpu().numpy(), ref["recv_count"])
+    assert np.array_equal(layout_range.cpu().numpy(), ref["layout_range"])
+
+
 def test_all_masked_and_duplicates(cuda_device):
     cfg = CONFIGS["tiny"].scaled(num_tokens=8 * 30, expert_alignment=4)
     wl = make_workload(cfg, 0)
