@@ -103,6 +103,27 @@ def test_quant_variants(quant, qs, rs, cuda_device):
     run_and_compare(cfg, 0, cuda_device)
 
 
+@pytest.mark.parametrize("quant,qs,H", [("fp8", 128, 16384), ("int8", 64, 24576), ("mxfp4", 32, 16384),
+                                        ("fp8", 512, 40960)])
+def test_group_quant_rows_of_several_passes(quant, qs, H, cuda_device):
+    """Group quantisation of rows longer than one pass of the group kernel
+    (512 threads x 16 channels = 8192 channels): 2, 3 and 5 passes per row,
+    with padding rows."""
+    cfg = CONFIGS["decode"].scaled(num_tokens=16 * 3, hidden=H, quant=quant, quant_size=qs, expert_alignment=4)
+    if quant != "mxfp4":
+        run_and_compare(cfg, 1, cuda_device)
+        return
+    wl = make_workload(cfg, 1)
+    x, ti, tw = to_dev(wl, cuda_device)
+    recv_x, recv_scales, _, _, h = ep.ep_dispatch(x, ti, tw, 4, quant, num_experts=cfg.num_experts,
+                                                  num_ranks=cfg.num_ranks, quant_size=qs)
+    s = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, 4)
+    n = s["num_recv_rows"]
+    ref_x, ref_s = oracle.dispatch_rows_mx(wl.x, s["dst_buffer_slot_idx"], quant, qs, num_rows=n)
+    assert np.array_equal(recv_x.contiguous().view(torch.uint8).cpu().numpy().reshape(n, -1), ref_x)
+    assert np.array_equal(recv_scales.contiguous().cpu().numpy(), ref_s)
+
+
 @pytest.mark.parametrize("quant,H", [("int8", 16384), ("fp8", 24576), ("int8", 65536)])
 def test_per_token_quant_large_hidden(quant, H, cuda_device):
     """Per-token quantisation of long rows: up to 1024 units of 16 channels
