@@ -5,7 +5,8 @@ hidden size, expert alignment, masking, x's magnitude, the number of rounds
 and the dispatch quantisation (none, FP8 / int8 with groups of 16-512 or per
 token, with or without power-of-two scales and UE8M0 bytes, MXFP4), then
 compares layout, slots, metadata, rows, codes, scales and the combine of
-seeded expert outputs.  Some cases also run the low-latency layout.
+seeded expert outputs (with and without a shared expert's row).  Some cases
+also run the low-latency layout.
 """
 import numpy as np
 import pytest
@@ -84,6 +85,15 @@ def test_random_configuration(i, cuda_device):
     h.check()
     ref_out = oracle.combine(y_np, s["dst_buffer_slot_idx"], wl.topk_weights, R, cfg.num_rounds)
     assert np.array_equal(u16(out), ref_out)
+    if i % 2 == 0:
+        # the same combine seeded with a shared expert's bf16 output
+        shared_np = make_y(T, H, i + 3)
+        shared = torch.from_numpy(shared_np.view(np.int16)).view(torch.bfloat16).to(dev)
+        out = ep.ep_combine(y, h, tw, shared=shared)
+        torch.cuda.synchronize()
+        h.check()
+        ref_sh = oracle.combine_rows_q(y_np, None, "none", 0, s["dst_buffer_slot_idx"], wl.topk_weights, shared_np)
+        assert np.array_equal(u16(out), ref_sh)
 
 
 @pytest.mark.parametrize("i", range(0, N_CASES, 3))
