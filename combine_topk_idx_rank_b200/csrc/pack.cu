@@ -306,6 +306,13 @@ __device__ __forceinline__ float finish_scale(float amax, float qmax, int round_
     return round_scale ? pow2_ceil_bits(s) : s;
 }
 
+// The routing kernel that this pack depends on stopped on its bounded wait:
+// the handle's rows and counts were not written, so nothing is packed (the
+// status word already holds EP_ERR_TIMEOUT).
+__device__ __forceinline__ bool routing_gave_up(const PackArgs& a) {
+    return *reinterpret_cast<const volatile int32_t*>(a.err) == EP_ERR_TIMEOUT;
+}
+
 // A destination row as the pack kernels use it: rows at or past the receive
 // capacity (a handle with foreign rows, or slots left stale by routing that
 // stopped on an error) are reported as EP_ERR_CAPACITY and dropped (-1).
@@ -332,6 +339,7 @@ template <int S>
 __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
     grid_dependency_wait();
     grid_launch_dependents();
+    if (routing_gave_up(a)) return;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* stage = smem;
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * chunk_bytes);
@@ -441,7 +449,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
                 const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, p);
                 const int64_t off = (int64_t)c * chunk_bytes;
                 const uint32_t bytes = (uint32_t)min((int64_t)chunk_bytes, row_bytes - off);
-                if (row < a.capacity) bulk_store(a.recv_x + row * row_bytes + off, stage, bytes);
+                if (row >= 0 && row < a.capacity) bulk_store(a.recv_x + row * row_bytes + off, stage, bytes);
             }
             bulk_commit();
         }
@@ -456,6 +464,7 @@ template <int VPT>
 __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
+    if (routing_gave_up(a)) return;
     __shared__ int s_slot[kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     const int tid = threadIdx.x;
@@ -488,7 +497,7 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
             }
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
-            if (row < a.capacity) {
+            if (row >= 0 && row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H * 2);
                 for (int v = tid; v < V; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
             }
@@ -509,6 +518,7 @@ template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_group(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
+    if (routing_gave_up(a)) return;
     __shared__ int s_slot[2][kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
@@ -605,7 +615,7 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
             }
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - n_tok);
-            if (row < a.capacity) {
+            if (row >= 0 && row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * row_bytes);
                 for (size_t v = tid; v < row_bytes / 16; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
                 zero_scales(a, row, nscales);
@@ -629,6 +639,7 @@ template <int QUANT, int UPT>
 __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
     grid_dependency_wait();
     grid_launch_dependents();
+    if (routing_gave_up(a)) return;
     __shared__ int s_slot[kMaxTopk];
     __shared__ float s_red[33];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
@@ -693,7 +704,7 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             }
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - a.n_tok_items);
-            if (row < a.capacity) {
+            if (row >= 0 && row < a.capacity) {
                 uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * a.H);
                 for (int v = tid; v < U; v += blockDim.x) st_v4(dst + v, make_uint4(0, 0, 0, 0));
                 if (tid == 0) zero_scales(a, row, 1);

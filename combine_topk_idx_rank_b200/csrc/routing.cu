@@ -20,27 +20,37 @@
 //      kernel).  CTA 0 writes the per-expert / per-rank
 //      outputs and the status word.
 // No sort, no global atomics except the barrier counter.
+#include <stdlib.h>
+
 #include "ep_internal.cuh"
 
 namespace ep {
 
 namespace {
 
-constexpr unsigned kBarrierSpinLimit = 1u << 24;   // x 64 ns sleeps
+constexpr unsigned long long kBarrierTimeoutNs = 2000000000ull;   // a grid barrier gives up after 2 s
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 // Grid-wide barrier over a counter that was zero at launch; `target` is
-// gridDim.x times the barrier's ordinal.  False if the bounded wait gave up.
+// gridDim.x times the barrier's ordinal.  False if the wait gave up (after
+// kBarrierTimeoutNs of the global timer).
 __device__ bool grid_barrier(unsigned* counter, unsigned target, int* s_flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         atomicAdd(counter, 1u);
         int ok = 1;
-        for (unsigned n = 0;; ++n) {
+        const unsigned long long t0 = global_ns();
+        for (;;) {
             unsigned v;
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
             if (v >= target) break;
-            if (n >= kBarrierSpinLimit) {
+            if (global_ns() - t0 > kBarrierTimeoutNs) {
                 ok = 0;
                 break;
             }
@@ -109,7 +119,9 @@ __device__ int block_exclusive_scan_E(const int* in, int* out, int E, int* s_war
 }  // namespace
 
 template <int KT>
-__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
+// stall > 0 (a test of the bounded wait only) raises the first barrier's
+// target past the number of CTAs, so that no CTA can pass it.
+__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a, unsigned stall) {
     grid_launch_dependents();   // the pack kernel may be scheduled; it waits for our results
     extern __shared__ int32_t smem[];
     const int E = a.E, K = KT > 0 ? KT : a.K, R = a.R, L = a.L;
@@ -227,7 +239,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         if (tid == 0) a.chunk_err[c] = *s_err;
         __syncthreads();
     }
-    if (!grid_barrier(a.barrier, (unsigned)G, s_flag)) {
+    if (!grid_barrier(a.barrier, (unsigned)G + stall, s_flag)) {
         if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
         return;
     }
@@ -442,7 +454,11 @@ cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_route<KT>, a);
+    // EP_TEST_STALL_BARRIER=1 in the environment makes the first grid barrier
+    // unreachable, for tests of the timeout path (EP_ERR_TIMEOUT after 2 s)
+    const char* stall_env = getenv("EP_TEST_STALL_BARRIER");
+    const unsigned stall = stall_env != nullptr && stall_env[0] == '1' ? 1u : 0u;
+    return cudaLaunchKernelEx(&cfg, k_route<KT>, a, stall);
 }
 
 }  // namespace

@@ -24,7 +24,11 @@
  *     receive capacity that is too small) are written to the device word
  *     `err`; read it with ep_read_error.  When *err != 0 the outputs are
  *     unspecified, but no kernel ever writes outside the buffers described
- *     here and none waits on anything.
+ *     here and none waits without a bound.
+ *   - The routing kernel's grid barriers give up after 2 s (EP_ERR_TIMEOUT);
+ *     the pack kernels of that call then write nothing.  For tests of that
+ *     path, EP_TEST_STALL_BARRIER=1 in the environment makes the first
+ *     barrier unreachable.
  *   - Sizes: T tokens (all logical ranks together), K top-k entries per
  *     token, E experts, R logical ranks, L = E / R local experts per rank,
  *     H hidden channels, A expert alignment.  Token t belongs to source rank
@@ -49,7 +53,8 @@ typedef enum {
     EP_ERR_BAD_EXPERT_ID = 2, /* some topk_idx entry is < -1 or >= E (device) */
     EP_ERR_CAPACITY = 3,      /* recv_capacity < rows needed (device) */
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
-    EP_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up */
+    EP_ERR_TIMEOUT = 5        /* a bounded device wait gave up (routing's grid barrier
+                                 waits at most 2 s); nothing is packed after it */
 } ep_status_t;
 
 typedef enum {
