@@ -171,3 +171,54 @@ def test_random_cached_dispatch_and_quantised_combine(i, cuda_device):
         ref_out = oracle.combine_rows_q(ref_x.reshape(n, -1), ref_s, cfg.quant, cfg.quant_size,
                                         s["dst_buffer_slot_idx"], wl.topk_weights, shared_np)
         assert np.array_equal(u16(out), ref_out)
+
+
+@pytest.mark.parametrize("i", range(0, N_CASES, 4))
+def test_random_error_paths(i, cuda_device):
+    """On the same draws: an out-of-range expert id is reported as
+    EP_ERR_BAD_EXPERT_ID (dispatch and layout call), and a receive capacity a
+    few rows short of what the routing needs is reported as EP_ERR_CAPACITY
+    with nothing written at or past the capacity."""
+    dev = cuda_device
+    cfg, ue8 = _draw(i)
+    T, H, K, E, R, A = (cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks,
+                        cfg.expert_alignment)
+    if T == 0:
+        pytest.skip("no tokens: no entry to corrupt, no row to overflow")
+    q = None if cfg.quant == "none" else cfg.quant
+    rng = np.random.default_rng(7000 + i)
+    wl = make_workload(cfg, seed=i)
+    kw = dict(num_experts=E, num_ranks=R, quant_size=cfg.quant_size, round_scale=cfg.round_scale,
+              num_rounds=cfg.num_rounds, scale_ue8m0=ue8)
+    need = oracle.slots(wl.topk_idx, wl.topk_weights, E, R, A)["num_recv_rows"]
+
+    bad = wl.topk_idx.copy()
+    bad[int(rng.integers(T)), int(rng.integers(K))] = int(rng.choice([E, E + 5, -2]))
+    x, _, tw = to_dev(wl, dev)
+    ti_bad = torch.from_numpy(bad).to(dev)
+    _, _, _, _, h = ep.ep_dispatch(x, ti_bad, tw, A, q, do_cpu_sync=False, **kw)
+    torch.cuda.synchronize()
+    assert h.read_error() == ep.EP_ERR_BAD_EXPERT_ID
+    with pytest.raises(ep.EPError) as e:
+        ep.ep_get_dispatch_layout(ti_bad, E, R)
+    assert e.value.status == ep.EP_ERR_BAD_EXPERT_ID
+
+    if need == 0:
+        return
+    cap = int(rng.integers(max(0, need - 40), need))
+    full = ep.alloc_dispatch_buffers(T, H, K, E, R, A, q, cfg.quant_size, cfg.num_rounds, recv_capacity=need + 64,
+                                     device=dev, scale_ue8m0=ue8)
+    tails = [full.recv_x, full.recv_topk_idx, full.recv_topk_weights, full.handle.recv_src_metadata]
+    if full.recv_scales is not None:
+        tails.append(full.recv_scales)
+    for t in tails:
+        t.view(torch.uint8).fill_(0xA5)
+    short = ep.DispatchBuffers(full.recv_x[:cap], None if full.recv_scales is None else full.recv_scales[:cap],
+                               full.recv_topk_idx[:cap], full.recv_topk_weights[:cap], full.handle, full.workspace,
+                               q, cfg.quant_size)
+    ti = torch.from_numpy(wl.topk_idx).to(dev)
+    ep.ep_dispatch(x, ti, tw, A, q, buffers=short, do_cpu_sync=False, **kw)
+    torch.cuda.synchronize()
+    assert full.handle.read_error() == ep.EP_ERR_CAPACITY
+    for t in tails:
+        assert torch.all(t[cap:].contiguous().view(torch.uint8) == 0xA5)
