@@ -214,7 +214,8 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
  * contents.  Padding rows are zeroed again.
  *   x            device bf16 [T,H] with the handle's T and H
  *   handle       filled by ep_dispatch (read only); its err word receives
- *                device errors of this call
+ *                device errors of this call (a handle whose err word already
+ *                holds EP_ERR_TIMEOUT from its routing is not packed)
  *   opts         quant, quant_size, round_scale, num_rounds and the optional
  *                pack events are used; expert_alignment is the handle's
  *   recv_x, recv_scales  as in ep_dispatch, handle->recv_capacity rows
