@@ -4,6 +4,10 @@ TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 benchmark's CPU-baseline leg, never by the product path.  The arithmetic lives
 in ep_oracle.c (plain C, single-threaded); this module only marshals numpy
 arrays.  It imports nothing from the CUDA package.
+
+``use_threads(n)`` with n > 1 routes the row functions (dispatch rows and
+combine) to the OpenMP build of the same source, which splits their token
+loops across n threads; every token's arithmetic is unchanged.
 """
 from __future__ import annotations
 
@@ -26,57 +30,86 @@ class OracleError(RuntimeError):
 
 
 _lib = None
+_lib_omp = None
+_threads = 1
 
 
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = C.CDLL(path)
-        p = C.c_void_p
-        i32, i64 = C.c_int32, C.c_int64
-        L.oracle_bf16_to_f32.argtypes = [C.c_uint16]
-        L.oracle_bf16_to_f32.restype = C.c_float
-        L.oracle_f32_to_bf16.argtypes = [C.c_float]
-        L.oracle_f32_to_bf16.restype = C.c_uint16
-        L.oracle_e4m3_to_f64.argtypes = [C.c_uint8]
-        L.oracle_e4m3_to_f64.restype = C.c_double
-        L.oracle_f32_to_e4m3.argtypes = [C.c_float]
-        L.oracle_f32_to_e4m3.restype = C.c_uint8
-        L.oracle_pow2_ceil.argtypes = [C.c_float]
-        L.oracle_pow2_ceil.restype = C.c_float
-        L.oracle_layout.argtypes = [p, i32, i32, i32, i32, p, p, p]
-        L.oracle_layout.restype = C.c_int
-        L.oracle_slots.argtypes = [p, p, i32, i32, i32, i32, i32, i64, p, p, p, p, p, p, p]
-        L.oracle_slots.restype = C.c_int
-        L.oracle_quantize_row.argtypes = [p, i32, i32, i32, i32, p, p]
-        L.oracle_quantize_row.restype = C.c_int
-        L.oracle_dispatch_rows.argtypes = [p, i32, i32, i32, p, i32, i32, i32, p, i64, p, p, i64]
-        L.oracle_dispatch_rows.restype = C.c_int
-        L.oracle_combine_rows.argtypes = [p, i64, i32, i32, i32, p, p, p, i64, p]
-        L.oracle_combine_rows.restype = C.c_int
-        L.oracle_round_tokens.argtypes = [i32, i32, i32, i32, p]
-        L.oracle_round_tokens.restype = i64
-        L.oracle_ll_slots.argtypes = [p, p, i32, i32, i32, i32, i32, p, p, p, p, p, p]
-        L.oracle_ll_slots.restype = C.c_int
-        L.oracle_combine_rows_q.argtypes = [p, p, i32, i32, i64, i32, i32, i32, p, p, p, p, i64, p]
-        L.oracle_combine_rows_q.restype = C.c_int
-        L.oracle_e2m1_to_f64.argtypes = [C.c_uint8]
-        L.oracle_e2m1_to_f64.restype = C.c_double
-        L.oracle_f32_to_e2m1.argtypes = [C.c_float]
-        L.oracle_f32_to_e2m1.restype = C.c_uint8
-        L.oracle_quantize_row_mx.argtypes = [p, i32, i32, i32, i32, i32, p, p]
-        L.oracle_quantize_row_mx.restype = C.c_int
-        L.oracle_dispatch_rows_mx.argtypes = [p, i32, i32, i32, p, i32, i32, i32, i32, p, i64, p, p, i64]
-        L.oracle_dispatch_rows_mx.restype = C.c_int
-        L.oracle_f32_to_e4m3_n.argtypes = [p, i64, p]
-        L.oracle_f32_to_e4m3_n.restype = None
-        L.oracle_f32_to_bf16_n.argtypes = [p, i64, p]
-        L.oracle_f32_to_bf16_n.restype = None
-        L.oracle_e4m3_to_f64_n.argtypes = [p, i64, p]
-        L.oracle_e4m3_to_f64_n.restype = None
-        _lib = L
+        _lib = _setup(C.CDLL(_build.build()))
     return _lib
+
+
+def _rowlib():
+    """The library the row functions call: the OpenMP build once use_threads(n > 1)."""
+    global _lib_omp
+    if _threads <= 1:
+        return lib()
+    if _lib_omp is None:
+        _lib_omp = _setup(C.CDLL(_build.build_omp()))
+    _lib_omp.oracle_threads(_threads)
+    return _lib_omp
+
+
+def use_threads(n: int) -> int:
+    """Row functions run on n threads (1 = the single-threaded build); returns n."""
+    global _threads
+    _threads = max(1, int(n))
+    return _rowlib().oracle_threads(0) if _threads > 1 else 1
+
+
+def threads() -> int:
+    return _threads
+
+
+def _setup(L):
+    """Declares the argument and result types of every oracle function."""
+    p = C.c_void_p
+    i32, i64 = C.c_int32, C.c_int64
+    L.oracle_bf16_to_f32.argtypes = [C.c_uint16]
+    L.oracle_bf16_to_f32.restype = C.c_float
+    L.oracle_f32_to_bf16.argtypes = [C.c_float]
+    L.oracle_f32_to_bf16.restype = C.c_uint16
+    L.oracle_e4m3_to_f64.argtypes = [C.c_uint8]
+    L.oracle_e4m3_to_f64.restype = C.c_double
+    L.oracle_f32_to_e4m3.argtypes = [C.c_float]
+    L.oracle_f32_to_e4m3.restype = C.c_uint8
+    L.oracle_pow2_ceil.argtypes = [C.c_float]
+    L.oracle_pow2_ceil.restype = C.c_float
+    L.oracle_layout.argtypes = [p, i32, i32, i32, i32, p, p, p]
+    L.oracle_layout.restype = C.c_int
+    L.oracle_slots.argtypes = [p, p, i32, i32, i32, i32, i32, i64, p, p, p, p, p, p, p]
+    L.oracle_slots.restype = C.c_int
+    L.oracle_quantize_row.argtypes = [p, i32, i32, i32, i32, p, p]
+    L.oracle_quantize_row.restype = C.c_int
+    L.oracle_dispatch_rows.argtypes = [p, i32, i32, i32, p, i32, i32, i32, p, i64, p, p, i64]
+    L.oracle_dispatch_rows.restype = C.c_int
+    L.oracle_combine_rows.argtypes = [p, i64, i32, i32, i32, p, p, p, i64, p]
+    L.oracle_combine_rows.restype = C.c_int
+    L.oracle_round_tokens.argtypes = [i32, i32, i32, i32, p]
+    L.oracle_round_tokens.restype = i64
+    L.oracle_ll_slots.argtypes = [p, p, i32, i32, i32, i32, i32, p, p, p, p, p, p]
+    L.oracle_ll_slots.restype = C.c_int
+    L.oracle_combine_rows_q.argtypes = [p, p, i32, i32, i64, i32, i32, i32, p, p, p, p, i64, p]
+    L.oracle_combine_rows_q.restype = C.c_int
+    L.oracle_e2m1_to_f64.argtypes = [C.c_uint8]
+    L.oracle_e2m1_to_f64.restype = C.c_double
+    L.oracle_f32_to_e2m1.argtypes = [C.c_float]
+    L.oracle_f32_to_e2m1.restype = C.c_uint8
+    L.oracle_quantize_row_mx.argtypes = [p, i32, i32, i32, i32, i32, p, p]
+    L.oracle_quantize_row_mx.restype = C.c_int
+    L.oracle_dispatch_rows_mx.argtypes = [p, i32, i32, i32, p, i32, i32, i32, i32, p, i64, p, p, i64]
+    L.oracle_dispatch_rows_mx.restype = C.c_int
+    L.oracle_f32_to_e4m3_n.argtypes = [p, i64, p]
+    L.oracle_f32_to_e4m3_n.restype = None
+    L.oracle_f32_to_bf16_n.argtypes = [p, i64, p]
+    L.oracle_f32_to_bf16_n.restype = None
+    L.oracle_e4m3_to_f64_n.argtypes = [p, i64, p]
+    L.oracle_e4m3_to_f64_n.restype = None
+    L.oracle_threads.argtypes = [C.c_int]
+    L.oracle_threads.restype = C.c_int
+    return L
 
 
 def _ptr(a: Optional[np.ndarray]):
@@ -200,7 +233,7 @@ def dispatch_rows(x, dst_buffer_slot_idx, quant: str = "none", quant_size: int =
     else:
         recv_x, recv_scales = out
         rows = recv_x.shape[0]
-    st = lib().oracle_dispatch_rows(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size,
+    st = _rowlib().oracle_dispatch_rows(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size,
                                     int(round_scale), _ptr(tok), tok.shape[0], _ptr(recv_x),
                                     _ptr(recv_scales), rows)
     if st:
@@ -218,7 +251,7 @@ def combine_rows(y, dst_buffer_slot_idx, topk_weights, tokens=None):
         tokens = np.arange(T, dtype=np.int32)
     tok = _c(tokens, np.int32)
     out = np.zeros((tok.shape[0], H), np.uint16)
-    st = lib().oracle_combine_rows(_ptr(ys), ys.shape[0], H, T, K, _ptr(dst), _ptr(tw), _ptr(tok),
+    st = _rowlib().oracle_combine_rows(_ptr(ys), ys.shape[0], H, T, K, _ptr(dst), _ptr(tw), _ptr(tok),
                                    tok.shape[0], _ptr(out))
     if st:
         raise OracleError(st, "combine_rows")
@@ -304,7 +337,7 @@ def combine_rows_q(y, y_scales, quant: str, quant_size: int, dst_buffer_slot_idx
         tokens = np.arange(T, dtype=np.int32)
     tok = _c(tokens, np.int32)
     out = np.zeros((tok.shape[0], H), np.uint16)
-    st = lib().oracle_combine_rows_q(_ptr(ys), _ptr(sc), QUANT[quant], quant_size, ys.shape[0], H, T, K,
+    st = _rowlib().oracle_combine_rows_q(_ptr(ys), _ptr(sc), QUANT[quant], quant_size, ys.shape[0], H, T, K,
                                      _ptr(dst), _ptr(tw), _ptr(sh), _ptr(tok), tok.shape[0], _ptr(out))
     if st:
         raise OracleError(st, "combine_rows_q")
@@ -358,7 +391,7 @@ def dispatch_rows_mx(x, dst_buffer_slot_idx, quant: str, quant_size: int, round_
     nb, sdt, ns = row_layout(H, quant, quant_size, scale_ue8m0)
     recv_x = np.zeros((rows, nb), np.uint8)
     recv_scales = None if sdt is None else np.zeros((rows, ns), sdt)
-    st = lib().oracle_dispatch_rows_mx(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size, int(round_scale),
+    st = _rowlib().oracle_dispatch_rows_mx(_ptr(xs), T, H, K, _ptr(dst), QUANT[quant], quant_size, int(round_scale),
                                        int(scale_ue8m0), _ptr(tok), tok.shape[0], _ptr(recv_x),
                                        _ptr(recv_scales), rows)
     if st:

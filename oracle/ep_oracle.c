@@ -6,6 +6,12 @@
  * compare the CUDA path against.  It shares no code, header, table or helper
  * with the CUDA library, and the product path never calls it.
  *
+ * The same source also builds with OpenMP (liboracle_omp.so): the loops over
+ * independent tokens in the row functions are then split across threads.
+ * Every token's arithmetic is the one written here either way; only which
+ * thread computes it changes.  The row functions report the largest status
+ * code that any token met.
+ *
  * What it computes, and where the pages define it:
  *
  *  - get_dispatch_layout: num_tokens_per_rank, num_tokens_per_expert and
@@ -282,39 +288,53 @@ int oracle_quantize_row(const uint16_t* x, int H, int quant, int quant_size, int
  * = x[t] (bf16 bits) or its quantisation, computed once per source token and
  * copied to each of its rows.  recv_x rows are H*esize bytes (esize 2 for bf16,
  * 1 for fp8/int8); recv_scales rows are H/quant_size floats (quantised only). */
+static int dispatch_token(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
+                          int quant, int quant_size, int round_scale, int t, uint8_t* recv_x,
+                          float* recv_scales, int64_t capacity, uint8_t* q, float* sc) {
+    int esize = (quant == OR_QUANT_NONE) ? 2 : 1;
+    int ns = (quant == OR_QUANT_NONE) ? 0 : H / quant_size;
+    if (t < 0 || t >= T) return OR_INVALID_ARG;
+    const uint16_t* xr = x + (int64_t)t * H;
+    if (quant != OR_QUANT_NONE) {
+        int st = oracle_quantize_row(xr, H, quant, quant_size, round_scale, q, sc);
+        if (st) return st;
+    }
+    for (int k = 0; k < K; ++k) {
+        int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+        if (row < 0) continue;
+        if (row >= capacity) return OR_CAPACITY;
+        uint8_t* dst = recv_x + row * H * esize;
+        if (quant == OR_QUANT_NONE) {
+            memcpy(dst, xr, (size_t)H * 2);
+        } else {
+            memcpy(dst, q, (size_t)H);
+            memcpy(recv_scales + row * ns, sc, sizeof(float) * ns);
+        }
+    }
+    return OR_OK;
+}
+
 int oracle_dispatch_rows(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
                          int quant, int quant_size, int round_scale,
                          const int32_t* tokens, int64_t n_tokens,
                          uint8_t* recv_x, float* recv_scales, int64_t capacity) {
     if (H < 1) return OR_INVALID_ARG;
-    int esize = (quant == OR_QUANT_NONE) ? 2 : 1;
     int ns = (quant == OR_QUANT_NONE) ? 0 : H / quant_size;
-    uint8_t* q = malloc((size_t)H);
-    float* sc = malloc(sizeof(float) * (size_t)(ns > 0 ? ns : 1));
-    for (int64_t i = 0; i < n_tokens; ++i) {
-        int t = tokens[i];
-        if (t < 0 || t >= T) { free(q); free(sc); return OR_INVALID_ARG; }
-        const uint16_t* xr = x + (int64_t)t * H;
-        if (quant != OR_QUANT_NONE) {
-            int st = oracle_quantize_row(xr, H, quant, quant_size, round_scale, q, sc);
-            if (st) { free(q); free(sc); return st; }
+    int st = OR_OK;
+#pragma omp parallel reduction(max : st)
+    {
+        uint8_t* q = malloc((size_t)H);
+        float* sc = malloc(sizeof(float) * (size_t)(ns > 0 ? ns : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            int s = dispatch_token(x, T, H, K, dst_buffer_slot_idx, quant, quant_size, round_scale, tokens[i],
+                                   recv_x, recv_scales, capacity, q, sc);
+            if (s > st) st = s;
         }
-        for (int k = 0; k < K; ++k) {
-            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
-            if (row < 0) continue;
-            if (row >= capacity) { free(q); free(sc); return OR_CAPACITY; }
-            uint8_t* dst = recv_x + row * H * esize;
-            if (quant == OR_QUANT_NONE) {
-                memcpy(dst, xr, (size_t)H * 2);
-            } else {
-                memcpy(dst, q, (size_t)H);
-                memcpy(recv_scales + row * ns, sc, sizeof(float) * ns);
-            }
-        }
+        free(q);
+        free(sc);
     }
-    free(q);
-    free(sc);
-    return OR_OK;
+    return st;
 }
 
 /* -------------------------------------------------------------- combine */
@@ -322,24 +342,32 @@ int oracle_dispatch_rows(const uint16_t* x, int T, int H, int K, const int32_t* 
 /* out[i] = bf16( fma chain over k = 0..K-1 with dst_buffer_slot_idx[t,k] >= 0 of
  * topk_weights[t,k] * y[slot] ), starting from +0.0f, for t = tokens[i].
  * out is [n_tokens, H] (compact, in list order). */
+static int combine_token(const uint16_t* y, int64_t y_rows, int H, int T, int K,
+                         const int32_t* dst_buffer_slot_idx, const float* topk_weights, int t, uint16_t* out_row) {
+    if (t < 0 || t >= T) return OR_INVALID_ARG;
+    for (int h = 0; h < H; ++h) {
+        float acc = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+            if (row < 0) continue;
+            if (row >= y_rows) return OR_CAPACITY;
+            acc = fmaf(topk_weights[(int64_t)t * K + k], oracle_bf16_to_f32(y[row * H + h]), acc);
+        }
+        out_row[h] = oracle_f32_to_bf16(acc);
+    }
+    return OR_OK;
+}
+
 int oracle_combine_rows(const uint16_t* y, int64_t y_rows, int H, int T, int K,
                         const int32_t* dst_buffer_slot_idx, const float* topk_weights,
                         const int32_t* tokens, int64_t n_tokens, uint16_t* out) {
+    int st = OR_OK;
+#pragma omp parallel for schedule(dynamic, 4) reduction(max : st)
     for (int64_t i = 0; i < n_tokens; ++i) {
-        int t = tokens[i];
-        if (t < 0 || t >= T) return OR_INVALID_ARG;
-        for (int h = 0; h < H; ++h) {
-            float acc = 0.0f;
-            for (int k = 0; k < K; ++k) {
-                int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
-                if (row < 0) continue;
-                if (row >= y_rows) return OR_CAPACITY;
-                acc = fmaf(topk_weights[(int64_t)t * K + k], oracle_bf16_to_f32(y[row * H + h]), acc);
-            }
-            out[i * H + h] = oracle_f32_to_bf16(acc);
-        }
+        int s = combine_token(y, y_rows, H, T, K, dst_buffer_slot_idx, topk_weights, tokens[i], out + i * H);
+        if (s > st) st = s;
     }
-    return OR_OK;
+    return st;
 }
 
 /* ------------------------------------------------------- long sequences */
@@ -426,34 +454,44 @@ int oracle_ll_slots(const int64_t* topk_idx, const float* topk_weights, int T, i
  * fma chain.  quant OR_QUANT_NONE reads bf16 y.  If `shared` is given (bf16
  * [T,H], a shared expert's output), the accumulator starts from shared[t]
  * instead of +0. */
+static int combine_token_q(const void* y, const float* y_scales, int quant, int quant_size, int64_t y_rows,
+                           int H, int T, int K, const int32_t* dst_buffer_slot_idx, const float* topk_weights,
+                           const uint16_t* shared, int t, uint16_t* out_row) {
+    int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
+    if (t < 0 || t >= T) return OR_INVALID_ARG;
+    for (int h = 0; h < H; ++h) {
+        float acc = shared ? oracle_bf16_to_f32(shared[(int64_t)t * H + h]) : 0.0f;
+        for (int k = 0; k < K; ++k) {
+            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+            if (row < 0) continue;
+            if (row >= y_rows) return OR_CAPACITY;
+            float v;
+            if (quant == OR_QUANT_NONE) {
+                v = oracle_bf16_to_f32(((const uint16_t*)y)[row * H + h]);
+            } else {
+                uint8_t c = ((const uint8_t*)y)[row * H + h];
+                float d = quant == OR_QUANT_FP8 ? (float)oracle_e4m3_to_f64(c) : (float)(int8_t)c;
+                v = d * y_scales[row * ns + h / quant_size];
+            }
+            acc = fmaf(topk_weights[(int64_t)t * K + k], v, acc);
+        }
+        out_row[h] = oracle_f32_to_bf16(acc);
+    }
+    return OR_OK;
+}
+
 int oracle_combine_rows_q(const void* y, const float* y_scales, int quant, int quant_size, int64_t y_rows,
                           int H, int T, int K, const int32_t* dst_buffer_slot_idx, const float* topk_weights,
                           const uint16_t* shared, const int32_t* tokens, int64_t n_tokens, uint16_t* out) {
     if (quant != OR_QUANT_NONE && (quant_size < 1 || H % quant_size != 0)) return OR_INVALID_ARG;
-    int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
+    int st = OR_OK;
+#pragma omp parallel for schedule(dynamic, 4) reduction(max : st)
     for (int64_t i = 0; i < n_tokens; ++i) {
-        int t = tokens[i];
-        if (t < 0 || t >= T) return OR_INVALID_ARG;
-        for (int h = 0; h < H; ++h) {
-            float acc = shared ? oracle_bf16_to_f32(shared[(int64_t)t * H + h]) : 0.0f;
-            for (int k = 0; k < K; ++k) {
-                int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
-                if (row < 0) continue;
-                if (row >= y_rows) return OR_CAPACITY;
-                float v;
-                if (quant == OR_QUANT_NONE) {
-                    v = oracle_bf16_to_f32(((const uint16_t*)y)[row * H + h]);
-                } else {
-                    uint8_t c = ((const uint8_t*)y)[row * H + h];
-                    float d = quant == OR_QUANT_FP8 ? (float)oracle_e4m3_to_f64(c) : (float)(int8_t)c;
-                    v = d * y_scales[row * ns + h / quant_size];
-                }
-                acc = fmaf(topk_weights[(int64_t)t * K + k], v, acc);
-            }
-            out[i * H + h] = oracle_f32_to_bf16(acc);
-        }
+        int s = combine_token_q(y, y_scales, quant, quant_size, y_rows, H, T, K, dst_buffer_slot_idx,
+                                topk_weights, shared, tokens[i], out + i * H);
+        if (s > st) st = s;
     }
-    return OR_OK;
+    return st;
 }
 
 /* ------------------------------------------------ MXFP4 and UE8M0 scales */
@@ -540,39 +578,72 @@ int oracle_quantize_row_mx(const uint16_t* x, int H, int quant, int quant_size, 
 /* oracle_dispatch_rows for every quantisation, including MXFP4 and UE8M0
  * scale bytes.  Row bytes: 2H (bf16), H (FP8 / int8), H/2 (MXFP4); scale
  * bytes per row: H/quant_size times 4 (fp32) or 1 (UE8M0, always for MXFP4). */
+static int dispatch_token_mx(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
+                             int quant, int quant_size, int round_scale, int scale_ue8m0, int t, uint8_t* recv_x,
+                             uint8_t* recv_scales, int64_t capacity, uint8_t* q, uint8_t* sc) {
+    int ue8 = (quant == OR_QUANT_MXFP4) || scale_ue8m0;
+    int64_t row_bytes = quant == OR_QUANT_NONE ? 2 * (int64_t)H : quant == OR_QUANT_MXFP4 ? H / 2 : H;
+    int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
+    int64_t scale_bytes = (int64_t)ns * (ue8 ? 1 : 4);
+    if (t < 0 || t >= T) return OR_INVALID_ARG;
+    const uint16_t* xr = x + (int64_t)t * H;
+    if (quant != OR_QUANT_NONE) {
+        int st = oracle_quantize_row_mx(xr, H, quant, quant_size, round_scale, scale_ue8m0, q, sc);
+        if (st) return st;
+    }
+    for (int k = 0; k < K; ++k) {
+        int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
+        if (row < 0) continue;
+        if (row >= capacity) return OR_CAPACITY;
+        if (quant == OR_QUANT_NONE) {
+            memcpy(recv_x + row * row_bytes, xr, (size_t)row_bytes);
+        } else {
+            memcpy(recv_x + row * row_bytes, q, (size_t)row_bytes);
+            memcpy(recv_scales + row * scale_bytes, sc, (size_t)scale_bytes);
+        }
+    }
+    return OR_OK;
+}
+
 int oracle_dispatch_rows_mx(const uint16_t* x, int T, int H, int K, const int32_t* dst_buffer_slot_idx,
                             int quant, int quant_size, int round_scale, int scale_ue8m0,
                             const int32_t* tokens, int64_t n_tokens, uint8_t* recv_x, uint8_t* recv_scales,
                             int64_t capacity) {
     if (H < 1) return OR_INVALID_ARG;
     int ue8 = (quant == OR_QUANT_MXFP4) || scale_ue8m0;
-    int64_t row_bytes = quant == OR_QUANT_NONE ? 2 * (int64_t)H : quant == OR_QUANT_MXFP4 ? H / 2 : H;
     int ns = quant == OR_QUANT_NONE ? 0 : H / quant_size;
     int64_t scale_bytes = (int64_t)ns * (ue8 ? 1 : 4);
-    uint8_t* q = malloc((size_t)H);
-    uint8_t* sc = malloc((size_t)(scale_bytes > 0 ? scale_bytes : 1));
     int st = OR_OK;
-    for (int64_t i = 0; i < n_tokens && st == OR_OK; ++i) {
-        int t = tokens[i];
-        if (t < 0 || t >= T) { st = OR_INVALID_ARG; break; }
-        const uint16_t* xr = x + (int64_t)t * H;
-        if (quant != OR_QUANT_NONE) {
-            st = oracle_quantize_row_mx(xr, H, quant, quant_size, round_scale, scale_ue8m0, q, sc);
-            if (st) break;
+#pragma omp parallel reduction(max : st)
+    {
+        uint8_t* q = malloc((size_t)H);
+        uint8_t* sc = malloc((size_t)(scale_bytes > 0 ? scale_bytes : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            int s = dispatch_token_mx(x, T, H, K, dst_buffer_slot_idx, quant, quant_size, round_scale, scale_ue8m0,
+                                      tokens[i], recv_x, recv_scales, capacity, q, sc);
+            if (s > st) st = s;
         }
-        for (int k = 0; k < K; ++k) {
-            int64_t row = dst_buffer_slot_idx[(int64_t)t * K + k];
-            if (row < 0) continue;
-            if (row >= capacity) { st = OR_CAPACITY; break; }
-            if (quant == OR_QUANT_NONE) {
-                memcpy(recv_x + row * row_bytes, xr, (size_t)row_bytes);
-            } else {
-                memcpy(recv_x + row * row_bytes, q, (size_t)row_bytes);
-                memcpy(recv_scales + row * scale_bytes, sc, (size_t)scale_bytes);
-            }
-        }
+        free(q);
+        free(sc);
     }
-    free(q);
-    free(sc);
     return st;
+}
+
+/* ------------------------------------------------------------- threads */
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads the row functions use: 1 in the plain build; in the OpenMP build,
+ * n > 0 sets the count and the current count is returned. */
+int oracle_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
 }
