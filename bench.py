@@ -15,8 +15,10 @@ problem (seed + rank) and there is no data-path collective: weak scaling.
 Timing: CUDA events on the launching stream, a barrier and a device sync on
 both sides of the timed region, max over ranks.
 
---impl reference times the CPU oracle (single-threaded C, unmodified) on the
-host cores on a bounded sample of the same workload.
+--impl reference times the CPU oracle (unmodified C; its OpenMP build on every
+host core) on bounded token samples of the same workload.
+
+--gpus N without a torchrun environment starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -69,13 +71,16 @@ def measured_hbm_peak():
 
 
 def algorithmic_bytes(cfg, counts, T, scale_ue8m0=False, combine_quant=False, low_latency=False):
-    """Minimum HBM bytes of one dispatch and one combine, from the actual counts.
+    """Minimum HBM bytes of the three kernels of one step, from the actual counts.
 
-    Dispatch: topk_idx read once, topk_weights read, x read once, every received
-    row written once (padding rows included) with its scales, recv_topk_idx,
-    recv_topk_weights, recv_src_metadata, and dst_buffer_slot_idx written.
-    Combine: dst_buffer_slot_idx and weights read, each unmasked y row read
-    once, out written once."""
+    route (k_route): topk_idx (int64) and topk_weights read once; the int32
+    copy of topk_idx and dst_buffer_slot_idx written; for every received row
+    (padding included) recv_topk_idx, recv_topk_weights and recv_src_metadata
+    written; the per-expert psum and counts written.
+    pack: x read once, dst_buffer_slot_idx read, every received row written
+    once (padding rows included) with its scales.
+    combine: dst_buffer_slot_idx and topk_weights read, each unmasked y row
+    read once, out written once."""
     H, K, A, E = cfg.hidden, cfg.num_topk, cfg.expert_alignment, cfg.num_experts
     counts = np.asarray(counts, np.int64)
     n = int(counts.sum())
@@ -83,13 +88,13 @@ def algorithmic_bytes(cfg, counts, T, scale_ue8m0=False, combine_quant=False, lo
     esize = {"none": 2.0, "fp8": 1.0, "int8": 1.0, "mxfp4": 0.5}[cfg.quant]
     nscales = 0 if cfg.quant == "none" else H // cfg.quant_size
     sbytes = 1 if (scale_ue8m0 or cfg.quant == "mxfp4") else 4
-    pack = int(T * H * 2 + n_al * H * esize + n_al * nscales * sbytes + n_al * (2 * K * 4 + 8) + T * K * (8 + 4 + 4))
-    layout = T * K * 8 + 4 * E * 4
+    route = int(T * K * (8 + 4 + 4 + 4) + n_al * (2 * K * 4 + 8) + 2 * E * 4)
+    pack = int(T * H * 2 + T * K * 4 + n_al * H * esize + n_al * nscales * sbytes)
     if combine_quant:       # y rows read as 1-byte codes with fp32 scales
         combine = T * K * 8 + n * (H + nscales * 4) + T * H * 2
     else:
         combine = T * K * 8 + n * H * 2 + T * H * 2
-    return {"layout": layout, "pack": pack, "combine": combine, "rows": n, "rows_aligned": n_al}
+    return {"route": route, "pack": pack, "combine": combine, "rows": n, "rows_aligned": n_al}
 
 
 def source_digest(files):
@@ -242,6 +247,30 @@ def barrier(world: int):
 
 # ------------------------------------------------------------------ our arm
 
+def config_dict(args, cfg, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    T, H, K, E, R = cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks
+    opt = {"mode": "full", "tokens": 0, "quant": None, "ue8m0": False, "combine_quant": False}
+    opt.update({k: getattr(args, k) for k in opt if hasattr(args, k)})
+    args = argparse.Namespace(workload=args.workload, **opt)
+    ll = args.mode == "ll"
+    q = None if cfg.quant == "none" else cfg.quant
+    cap = E * R * (T // R) if ll else T * K + E * (cfg.expert_alignment - 1)
+    ebytes = 2 if q is None else (0.5 if q == "mxfp4" else 1)
+    return {"workload": WORKLOAD_DESC[args.workload] + (f" (scaled to {T} tokens)" if args.tokens else "")
+            + (" — cached dispatch (routing reused from the handle)" if args.mode == "cached" else "")
+            + (" — low-latency fixed-capacity layout" if ll else "")
+            + (f" — dispatch {cfg.quant} g{cfg.quant_size}{' ue8m0 bytes' if args.ue8m0 else ''}"
+               if args.quant or args.ue8m0 else "")
+            + (" — combine reads the quantised rows" if args.combine_quant else ""),
+            "name": args.workload, "mode": args.mode, "tokens": T, "hidden": H,
+            "num_experts": E, "num_ranks": R, "topk": K, "expert_alignment": cfg.expert_alignment,
+            "quant": cfg.quant, "num_rounds": cfg.num_rounds,
+            "parallelism": f"{world} independent EP problems",
+            "l2": "no flush: inputs larger than L2 (x %.0f MB, recv_x/y up to %.0f MB each)" % (
+                T * H * 2 / 1e6, cap * H * ebytes / 1e6)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -285,51 +314,39 @@ def run_ours(args):
         g.manual_seed(1234 + rank)
         y, y_scales = torch.randn((cap, H), generator=g, device=dev, dtype=torch.bfloat16), None
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for row in ev:               # create the events before handing them to the library
-        for e in row:
-            e.record()
-    torch.cuda.synchronize()
-
     if args.mode == "cached":       # routing computed once; every step re-packs with the handle
         ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
                        quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
                        do_cpu_sync=False, buffers=bufs)
 
-    # the kernel split is taken on every `every`-th timed step only: an event
-    # recorded between two kernels costs a few microseconds of stream time and
-    # stops the programmatic launch overlap of the kernels it separates
-    every = max(1, min(10, args.steps // 20))
-    sampled = [i for i in range(args.steps) if i % every == 0]
-
-    def step(i=None, x=x, ti=ti, tw=tw, out=out):
-        if i is not None and i % every:
-            i = None
-        evs = None if i is None else (ev[i][0], ev[i][1])
+    def step(evs=None, x=x, ti=ti, tw=tw, out=out):
+        """One dispatch + combine.  evs = four recorded events for the
+        per-kernel split (step start, pack begin, pack end, combine end), or
+        None: then nothing is recorded between the kernels."""
+        if evs is not None:
+            evs[0].record()
+        pev = None if evs is None else (evs[1], evs[2])
         if args.mode == "cached":
             ep.ep_dispatch(x, quant=q, quant_size=cfg.quant_size, round_scale=cfg.round_scale,
-                           num_rounds=cfg.num_rounds, buffers=bufs, events=evs, handle=bufs.handle,
+                           num_rounds=cfg.num_rounds, buffers=bufs, events=pev, handle=bufs.handle,
                            scale_ue8m0=ue8)
         elif ll:
             ep.ep_dispatch_low_latency(x, ti, tw, M, E, R, q, quant_size=cfg.quant_size,
                                        round_scale=cfg.round_scale, workspace=bufs.workspace, buffers=ll_bufs,
-                                       scale_ue8m0=ue8, events=evs)
+                                       scale_ue8m0=ue8, events=pev)
         else:
             ep.ep_dispatch(x, ti, tw, cfg.expert_alignment, q, num_experts=E, num_ranks=R,
                            quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
-                           do_cpu_sync=False, buffers=bufs, events=evs, scale_ue8m0=ue8)
-        if i is not None:
-            ev[i][2].record()
+                           do_cpu_sync=False, buffers=bufs, events=pev, scale_ue8m0=ue8)
         # y: the experts' outputs, produced on the device (random bf16, or the
         # received codes themselves with --combine-quant)
         ep.ep_combine(y, bufs.handle, tw, out=out, y_scales=y_scales, quant_size=cfg.quant_size)
-        if i is not None:
-            ev[i][3].record()
+        if evs is not None:
+            evs[3].record()
         return out
 
-    sampler = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)
-                           if str(torch.cuda.get_device_properties(dev).uuid).startswith("GPU-")
-                           else "GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     sampler.start()
     time.sleep(0.5)
     for _ in range(args.warmup):
@@ -338,23 +355,40 @@ def run_ours(args):
     bufs.handle.check()
     counts = bufs.handle.num_recv_tokens_per_expert.cpu().numpy()
 
+    # ------------------------------------------------- headline timed region
+    # K steps back to back with nothing recorded between the kernels, so the
+    # programmatic launch overlap of neighbouring kernels is the caller's
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
-    for i in range(args.steps):
-        step(i)
+    for _ in range(args.steps):
+        step()
     stop.record()
     torch.cuda.synchronize()
     barrier(world)
     t_wall1 = time.time()
     sampler.stop()
-    elapsed_ms = start.elapsed_time(stop)
-    pack_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in sampled) / len(sampled)
-    combine_ms = sum(ev[i][2].elapsed_time(ev[i][3]) for i in sampled) / len(sampled)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
 
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    # --------------------------------------------- per-kernel split (separate)
+    # events around each kernel of every step of a separate loop; an event
+    # between two kernels stops their launch overlap, so this loop runs a
+    # little slower than the headline one and is used for the split only
+    n_split = max(3, min(args.steps, 50))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_split)]
+    for row in ev:               # create the events before handing them to the library
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    for i in range(n_split):
+        step(ev[i])
+    torch.cuda.synchronize()
+    route_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(n_split))
+    pack_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(n_split))
+    combine_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(n_split))
+    split_step_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][3]) for i in range(n_split))
 
     # ------------------------------------------------------------ end to end
     e2e_steps = max(3, min(args.steps, 20))
@@ -418,10 +452,9 @@ def run_ours(args):
 
     ab = algorithmic_bytes(cfg, counts, T, ue8, args.combine_quant, ll)
     if args.mode == "cached":
-        ab["layout"] = 0
-        ab["pack"] -= T * cfg.num_topk * 8 + ab["rows_aligned"] * (2 * cfg.num_topk * 4 + 8)   # no routing / metadata
+        ab["route"] = 0
     ms_per_step = elapsed_ms / args.steps
-    step_bytes = ab["layout"] + ab["pack"] + ab["combine"]
+    step_bytes = ab["route"] + ab["pack"] + ab["combine"]
     value = job_tokens_per_s(world, T, ms_per_step)
     gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
@@ -430,7 +463,8 @@ def run_ours(args):
     if pack_ms >= combine_ms:
         dom, dom_bytes, dom_gbs, dom_ms = "k_pack", ab["pack"] / cfg.num_rounds, pack_gbs, pack_ms / cfg.num_rounds
     else:
-        dom, dom_bytes, dom_gbs, dom_ms = "k_combine", ab["combine"] / cfg.num_rounds, combine_gbs, combine_ms / cfg.num_rounds
+        dom, dom_bytes, dom_gbs, dom_ms = ("k_combine", ab["combine"] / cfg.num_rounds, combine_gbs,
+                                           combine_ms / cfg.num_rounds)
     clocks = sampler.summary(t_wall0, t_wall1)
     default_launch = (args.mode == "full" and not args.quant and not args.ue8m0 and not args.combine_quant
                       and not args.tokens)
@@ -442,25 +476,20 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q is None else f"bf16->{q}",
         "data": "synthetic (seeded numpy PCG64; no dataset, no weights)",
-        "config": {"workload": WORKLOAD_DESC[args.workload] + (f" (scaled to {T} tokens)" if args.tokens else "")
-                   + (" — cached dispatch (routing reused from the handle)" if args.mode == "cached" else "")
-                   + (" — low-latency fixed-capacity layout" if ll else "")
-                   + (f" — dispatch {cfg.quant} g{cfg.quant_size}{' ue8m0 bytes' if ue8 else ''}" if args.quant or ue8 else "")
-                   + (" — combine reads the quantised rows" if args.combine_quant else ""),
-                   "name": args.workload, "mode": args.mode, "tokens": T, "hidden": H,
-                   "num_experts": E, "num_ranks": R, "topk": K, "expert_alignment": cfg.expert_alignment,
-                   "quant": cfg.quant, "num_rounds": cfg.num_rounds, "parallelism": f"{world} independent EP problems",
-                   "l2": "inputs larger than L2 (x %.0f MB, recv_x/y %.0f MB each)" % (
-                       T * H * 2 / 1e6, cap * H * (2 if q is None else 1) / 1e6)},
+        "config": config_dict(args, cfg, world),
         "hbm": {"achieved_gbs": round(gbs, 1), "algorithmic_bytes_per_step": step_bytes,
                 "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "frac_of_measured": round(gbs / peak, 4),
-                "measured_peak_gbs": peak, "rows": ab["rows"], "rows_aligned": ab["rows_aligned"]},
-        "kernels": {"pack_ms": round(pack_ms, 5), "pack_gbs": round(pack_gbs, 1),
+                "measured_peak_gbs": peak, "rows": ab["rows"], "rows_aligned": ab["rows_aligned"],
+                "bytes": {"route": ab["route"], "pack": ab["pack"], "combine": ab["combine"]}},
+        "kernels": {"route_ms": round(route_ms, 5), "pack_ms": round(pack_ms, 5), "pack_gbs": round(pack_gbs, 1),
                     "combine_ms": round(combine_ms, 5), "combine_gbs": round(combine_gbs, 1),
-                    "routing_and_gaps_ms": round(ms_per_step - pack_ms - combine_ms, 5),
-                    "split_steps": len(sampled), "split_every": every},
+                    "split_steps": n_split, "split_step_ms": round(split_step_ms, 5),
+                    "note": "per-kernel CUDA events from a separate loop after the timed one; route_ms is "
+                            "the memset + routing kernel up to the pack's start"},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak, "unit": "GB/s",
                      "peak_kind": peak_kind, "frac": round(dom_gbs / peak, 4),
+                     "frac_of_8tbs": round(dom_gbs / NOMINAL_HBM_GBS, 4),
+                     "step_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
                      "algorithmic_bytes_per_launch": int(dom_bytes), "launch_ms": round(dom_ms, 5),
                      # the capture holds the workload's default launch only
                      "traffic": traffic_for(dom, args.workload) if default_launch else None},
@@ -471,7 +500,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, wl, budget_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(cfg, wl, step_bytes / T, budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(result), flush=True)
     barrier(world)
@@ -481,97 +510,161 @@ def run_ours(args):
 
 # ------------------------------------------------------------ oracle (CPU)
 
-def cpu_baseline(cfg, wl, budget_s=15.0, quick=False):
-    """Times the oracle as it stands, single-threaded, on this host: the slot
-    assignment over the whole routing, plus dispatch rows and combine for a
-    sample of tokens; reports the projected throughput of the full workload."""
-    import oracle
-    from combine_topk_idx_rank_b200.workloads import make_y
-    T, H = cfg.num_tokens, cfg.hidden
-    t0 = time.perf_counter()
-    s = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, cfg.expert_alignment)
-    t_slots = time.perf_counter() - t0
-    pool = 8192
-    dst = s["dst_buffer_slot_idx"]
-    pdst = np.where(dst >= 0, dst % pool, -1).astype(np.int32)
-    ypool = make_y(pool, H, 7)
-    # calibrate on a few tokens, then size the sample to the budget
-    rng = np.random.default_rng(0)
-    order = rng.permutation(T).astype(np.int32)
-    done, t_rows, used = 0, 0.0, 0
-    batch = 64
-    while True:
-        tok = order[used:used + batch]
-        if tok.size == 0:
-            break
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleSampler:
+    """Runs the oracle, as it stands, on token samples of a workload: one
+    sample = a smaller problem of the same shape (the same number of tokens
+    from every source rank, their routing and rows), through slot assignment,
+    dispatch rows and combine.  Rows are mapped into a pool of 8192 rows so
+    that memory stays bounded; each token's arithmetic is unchanged."""
+
+    POOL = 8192
+
+    def __init__(self, cfg, wl, seed=0):
+        from combine_topk_idx_rank_b200.workloads import make_y
+        self.cfg, self.wl = cfg, wl
+        self.ypool = make_y(self.POOL, cfg.hidden, 7)
+        self.rng = np.random.default_rng(seed)
+
+    def tokens(self, per_rank):
+        cfg = self.cfg
+        tpr = cfg.num_tokens // cfg.num_ranks
+        per_rank = max(1, min(tpr, per_rank))
+        picks = [r * tpr + np.sort(self.rng.choice(tpr, size=per_rank, replace=False))
+                 for r in range(cfg.num_ranks)]
+        return np.concatenate(picks).astype(np.int64)
+
+    def run(self, tok):
+        """Seconds the oracle takes for the sample `tok`."""
+        import oracle
+        cfg, wl = self.cfg, self.wl
+        idx, w, x = wl.topk_idx[tok], wl.topk_weights[tok], wl.x[tok]
         t0 = time.perf_counter()
-        oracle.dispatch_rows(wl.x, pdst, cfg.quant, cfg.quant_size, cfg.round_scale, tokens=tok, num_rows=pool)
-        oracle.combine_rows(ypool, pdst, wl.topk_weights, tokens=tok)
-        t_rows += time.perf_counter() - t0
-        used += tok.size
-        if t_rows + t_slots >= budget_s or quick:
-            break
-        batch = min(4096, batch * 2)
-    per_tok = t_rows / used
-    proj = t_slots + per_tok * T
-    return {"value": round(T / proj, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"slot assignment over all {T} tokens ({t_slots:.2f} s) + dispatch rows and combine "
-                      f"of {used} random tokens ({t_rows:.2f} s; rows mapped into a {pool}-row pool); "
-                      f"value = {T} / projected full-workload time",
-            "seconds": round(t_slots + t_rows, 2)}
+        s = oracle.slots(idx, w, cfg.num_experts, cfg.num_ranks, cfg.expert_alignment)
+        dst = s["dst_buffer_slot_idx"]
+        pdst = np.where(dst >= 0, dst % self.POOL, -1).astype(np.int32)
+        oracle.dispatch_rows(x, pdst, cfg.quant, cfg.quant_size, cfg.round_scale, num_rows=self.POOL)
+        oracle.combine_rows(self.ypool, pdst, w)
+        return time.perf_counter() - t0
+
+    def calibrate(self):
+        """Seconds per token, from a sample of 8 tokens per rank."""
+        tok = self.tokens(8)
+        self.run(tok)
+        return self.run(tok) / tok.size
+
+
+def cpu_baseline(cfg, wl, bytes_per_token, budget_s=12.0):
+    """The oracle timed on this host's cores: the single-threaded build on one
+    core, then the OpenMP build of the same source on every core in
+    sched_getaffinity, each on measured token samples (no projection)."""
+    import oracle
+    smp = OracleSampler(cfg, wl)
+    res = {}
+    for label, n in (("one_core", 1), ("all_cores", host_cores())):
+        used = oracle.use_threads(n)
+        per_tok = smp.calibrate()
+        per_rank = int(max(1, (budget_s / 2 / 3) / per_tok / cfg.num_ranks))
+        secs, toks = 0.0, 0
+        for _ in range(3):
+            tok = smp.tokens(per_rank)
+            secs += smp.run(tok)
+            toks += tok.size
+        res[label] = {"value": round(toks / secs, 2), "cores": used, "tokens": toks, "seconds": round(secs, 2),
+                      "gbs": round(toks / secs * bytes_per_token / 1e9, 4)}
+    oracle.use_threads(1)
+    allc, one = res["all_cores"], res["one_core"]
+    return {"value": allc["value"], "unit": UNIT, "cores": allc["cores"], "kind": "oracle",
+            "gbs": allc["gbs"], "one_core": one,
+            "sample": f"3 samples of {allc['tokens'] // 3} tokens (the same number from each of the "
+                      f"{cfg.num_ranks} ranks, with their routing) through the oracle's slot assignment, "
+                      f"dispatch rows and combine; all cores ({allc['cores']} threads, OpenMP build of the "
+                      f"same source) {allc['seconds']} s; one core {one['value']} tokens/s over "
+                      f"{one['tokens']} tokens ({one['seconds']} s); measured, not projected"}
 
 
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:       # under torchrun only rank 0 times the oracle
         return
+    import oracle
     cfg = workload_config(args)
     wl = make_workload(cfg, seed=args.seed)
-    import oracle
-    from combine_topk_idx_rank_b200.workloads import make_y
-    T, H = cfg.num_tokens, cfg.hidden
-    pool = 8192
-    ypool = make_y(pool, H, 7)
-    budget = args.ref_seconds
-    # per step: the slot assignment is done once per step only if it fits the
-    # step budget; otherwise once up front and charged pro rata per token
-    t0 = time.perf_counter()
-    s = oracle.slots(wl.topk_idx, wl.topk_weights, cfg.num_experts, cfg.num_ranks, cfg.expert_alignment)
-    t_slots = time.perf_counter() - t0
-    dst = s["dst_buffer_slot_idx"]
-    pdst = np.where(dst >= 0, dst % pool, -1).astype(np.int32)
-    t0 = time.perf_counter()
-    cal = np.arange(32, dtype=np.int32)
-    oracle.dispatch_rows(wl.x, pdst, cfg.quant, cfg.quant_size, cfg.round_scale, tokens=cal, num_rows=pool)
-    oracle.combine_rows(ypool, pdst, wl.topk_weights, tokens=cal)
-    per_tok = (time.perf_counter() - t0) / 32
+    T = cfg.num_tokens
+    cores = host_cores()
+    used = oracle.use_threads(cores)
+    smp = OracleSampler(cfg, wl, seed=args.seed)
+    per_tok = smp.calibrate()
     n_steps = args.steps + args.warmup
-    per_step_tokens = int(max(1, min(T, (budget / n_steps) / per_tok)))
-    rng = np.random.default_rng(args.seed)
-    times = []
+    per_rank = int(max(1, (args.ref_seconds / n_steps) / per_tok / cfg.num_ranks))
+    times, toks = [], []
     for i in range(n_steps):
-        tok = np.sort(rng.choice(T, size=per_step_tokens, replace=False)).astype(np.int32)
-        t0 = time.perf_counter()
-        oracle.dispatch_rows(wl.x, pdst, cfg.quant, cfg.quant_size, cfg.round_scale, tokens=tok, num_rows=pool)
-        oracle.combine_rows(ypool, pdst, wl.topk_weights, tokens=tok)
-        dt = time.perf_counter() - t0
+        tok = smp.tokens(per_rank)
+        dt = smp.run(tok)
         if i >= args.warmup:
             times.append(dt)
-    per_tok = sum(times) / (len(times) * per_step_tokens)
-    proj_s = t_slots + per_tok * T
-    value = T / proj_s
-    sample = (f"each step: dispatch rows + combine of {per_step_tokens} random tokens (rows mapped into a "
-              f"{pool}-row pool); slot assignment over all {T} tokens timed once ({t_slots:.2f} s) and "
-              f"charged pro rata; value = {T} / projected full-workload time")
+            toks.append(tok.size)
+    oracle.use_threads(1)
+    value = sum(toks) / sum(times)
+    ms_per_step = 1e3 * sum(times) / len(times)
+    per_step_tokens = toks[0]
+    sample = (f"each step: the oracle (OpenMP build, {used} threads) on {per_step_tokens} tokens "
+              f"({per_step_tokens // cfg.num_ranks} from each of the {cfg.num_ranks} ranks, with their routing): "
+              f"slot assignment, dispatch rows and combine (rows mapped into an {OracleSampler.POOL}-row pool); "
+              f"value = measured tokens / measured seconds")
     res = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(proj_s * 1e3, 3), "higher_is_better": True,
+           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.quant == "none" else f"bf16->{cfg.quant}",
-           "data": "synthetic (seeded numpy PCG64)", "impl": "reference",
-           "config": {"workload": WORKLOAD_DESC[args.workload], "name": args.workload},
-           "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+           "data": "synthetic (seeded numpy PCG64; no dataset, no weights)", "impl": "reference",
+           "config": config_dict(args, cfg, world),
+           "tokens_per_step": per_step_tokens,
+           "projected_full_workload_ms": round(1e3 * T / value, 1),
+           "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": used, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
+
+
+# ------------------------------------------------------------- launcher
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv, timeout_s: float = 3600.0) -> int:
+    """Starts n copies of this script, one per GPU, with the environment
+    torchrun gives (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR 127.0.0.1,
+    MASTER_PORT); rank 0's output is this process's output.  Returns the
+    first non-zero exit code, else 0."""
+    port = free_port()
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__), *argv], env=env,
+                                      stdout=None if r == 0 else subprocess.DEVNULL))
+    rc = 0
+    deadline = time.time() + timeout_s
+    for p in procs:
+        try:
+            code = p.wait(timeout=max(1.0, deadline - time.time()))
+        except subprocess.TimeoutExpired:
+            for q in procs:
+                if q.poll() is None:
+                    q.kill()
+            code = 124
+        if code and not rc:
+            rc = code
+    return rc
 
 
 def main(argv=None):
@@ -591,12 +684,16 @@ def main(argv=None):
     p.add_argument("--ue8m0", action="store_true", help="power-of-two scales stored as UE8M0 bytes")
     p.add_argument("--combine-quant", action="store_true",
                    help="combine reads the FP8 / int8 received rows (identity experts) instead of bf16 y")
-    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the cpu_baseline sample")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the cpu_baseline samples")
     p.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the --impl reference run")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    argv = sys.argv[1:] if argv is None else list(argv)
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU, as torchrun would start them
+        raise SystemExit(launch_ranks(args.gpus, argv))
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libep.so")
 OBJDIR = os.path.join(HERE, "_build")
 SOURCES = ["routing.cu", "pack.cu", "combine.cu", "ep_api.cu", "ep_noalloc.cu"]
-HEADERS = ["ep_internal.cuh", os.path.join("..", "..", "include", "ep.h")]
+HEADERS = ["ep_internal.cuh", os.path.join("..", "..", "include", "ep.h"),
+           os.path.join("..", "..", "include", "ep_testing.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -4,6 +4,7 @@
 #include <stdio.h>
 
 #include "ep_internal.cuh"
+#include "../../include/ep_testing.h"
 
 namespace ep {
 
@@ -139,10 +140,14 @@ const char* ep_status_string(ep_status_t s) {
     return "unknown status";
 }
 
-ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E,
-                                   int32_t R, int32_t* num_tokens_per_rank,
-                                   int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
-                                   int32_t* err, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The layout call; stall > 0 only from the test entry point.
+ep_status_t layout_impl(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E, int32_t R,
+                        int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                        int32_t* err, void* ws, size_t ws_bytes, void* stream, unsigned stall) {
     if (!sizes_ok(T, K, E, R) || err == nullptr || ws == nullptr) return EP_ERR_INVALID_ARG;
     if (T > 0 && topk_idx == nullptr) return EP_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(T, K, E, R);
@@ -153,16 +158,17 @@ ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K
     r.num_tokens_per_expert = num_tokens_per_expert;
     r.num_tokens_per_rank = num_tokens_per_rank;
     r.err_out = err;
+    r.stall = stall;
     return cuda_status(launch_route(r, static_cast<cudaStream_t>(stream)));
 }
 
-ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
-                        const float* topk_weights, int32_t K, int32_t E, int32_t R,
-                        const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
-                        int32_t* recv_topk_idx, float* recv_topk_weights,
-                        int64_t recv_capacity, ep_handle_t* h,
-                        int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
-                        uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream) {
+// Dispatch; stall > 0 only from the test entry point.
+ep_status_t dispatch_impl(const void* x, int32_t T, int32_t H, const int64_t* topk_idx, const float* topk_weights,
+                          int32_t K, int32_t E, int32_t R, const ep_dispatch_opts_t* opts, void* recv_x,
+                          float* recv_scales, int32_t* recv_topk_idx, float* recv_topk_weights,
+                          int64_t recv_capacity, ep_handle_t* h, int32_t* num_tokens_per_rank,
+                          int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank, void* ws, size_t ws_bytes,
+                          void* stream, unsigned stall) {
     if (!sizes_ok(T, K, E, R) || opts == nullptr || h == nullptr) return EP_ERR_INVALID_ARG;
     if (H < 8 || H > 65536 || H % 8 != 0) return EP_ERR_INVALID_ARG;
     const int A = opts->expert_alignment;
@@ -211,10 +217,55 @@ ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk
     r.num_tokens_per_rank = num_tokens_per_rank;
     r.cumulative = opts->cumulative_local_expert_recv_stats;
     r.err_out = h->err;
+    r.stall = stall;
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, recv_capacity, h,
                               st);
+}
+
+}  // namespace
+
+extern "C" {
+
+ep_status_t ep_get_dispatch_layout(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E,
+                                   int32_t R, int32_t* num_tokens_per_rank,
+                                   int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                                   int32_t* err, void* ws, size_t ws_bytes, void* stream) {
+    return layout_impl(topk_idx, T, K, E, R, num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank, err,
+                       ws, ws_bytes, stream, 0);
+}
+
+ep_status_t ep_dispatch(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                        const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                        const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                        int32_t* recv_topk_idx, float* recv_topk_weights,
+                        int64_t recv_capacity, ep_handle_t* h,
+                        int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                        uint8_t* is_token_in_rank, void* ws, size_t ws_bytes, void* stream) {
+    return dispatch_impl(x, T, H, topk_idx, topk_weights, K, E, R, opts, recv_x, recv_scales, recv_topk_idx,
+                         recv_topk_weights, recv_capacity, h, num_tokens_per_rank, num_tokens_per_expert,
+                         is_token_in_rank, ws, ws_bytes, stream, 0);
+}
+
+ep_status_t ep_testing_get_dispatch_layout_stalled(const int64_t* topk_idx, int32_t T, int32_t K, int32_t E,
+                                                   int32_t R, int32_t* num_tokens_per_rank,
+                                                   int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                                                   int32_t* err, void* ws, size_t ws_bytes, void* stream) {
+    return layout_impl(topk_idx, T, K, E, R, num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank, err,
+                       ws, ws_bytes, stream, 1);
+}
+
+ep_status_t ep_testing_dispatch_stalled(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,
+                                        const float* topk_weights, int32_t K, int32_t E, int32_t R,
+                                        const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
+                                        int32_t* recv_topk_idx, float* recv_topk_weights, int64_t recv_capacity,
+                                        ep_handle_t* h, int32_t* num_tokens_per_rank,
+                                        int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank, void* ws,
+                                        size_t ws_bytes, void* stream) {
+    return dispatch_impl(x, T, H, topk_idx, topk_weights, K, E, R, opts, recv_x, recv_scales, recv_topk_idx,
+                         recv_topk_weights, recv_capacity, h, num_tokens_per_rank, num_tokens_per_expert,
+                         is_token_in_rank, ws, ws_bytes, stream, 1);
 }
 
 ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const int64_t* topk_idx,

@@ -100,6 +100,9 @@ struct RouteArgs {
     int32_t* chunk_hist;
     int32_t* chunk_rcnt;
     int32_t* chunk_err;
+    // > 0 only from the test entry points: raises the first grid barrier's
+    // target past the number of CTAs, so that no CTA can pass it
+    unsigned stall;
 };
 
 struct PackArgs {

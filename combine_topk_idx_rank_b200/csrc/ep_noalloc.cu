@@ -16,8 +16,13 @@
 //     library, until the process exits.  Sizes whose scratch would not fit are
 //     rejected with EP_ERR_INVALID_ARG and a message on stderr; nothing runs.
 //   - The first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress, with that device current) and caches it; make
-//     that first call before any stream capture.
+//     (cudaGetSymbolAddress, with that device current) and caches it beside
+//     the ID of the device's current CUDA context; make that first call
+//     before any stream capture.  A later call in another context of that
+//     device (after cudaDeviceReset, or with the primary context released
+//     and created again) finds a different context ID and looks the address
+//     up again, so a stale address from a destroyed context is never used;
+//     that call, too, should come before any stream capture.
 //   - All calls share the one array per device and it keeps the last call's
 //     contents.  Dispatch rewrites every part of the scratch it reads in each
 //     call (and clears its barrier counter itself), so nothing needs clearing
@@ -25,6 +30,7 @@
 //     streams, or two host threads) race on the array and corrupt each other;
 //     serialise them on one stream.
 //   - No cudaMalloc, cudaFree or allocating library routine is called.
+#include <cuda.h>   // CUcontext / CUresult types; the driver calls are resolved at run time
 #include <mutex>
 #include <stdio.h>
 
@@ -38,11 +44,47 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_dispatch_scratch[kScratchBytes];
 
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};   // device address of g_dispatch_scratch, per device
+struct ScratchAddr {
+    unsigned long long ctx_id;   // ID of the context the address belongs to (0 = none yet)
+    void* addr;                  // device address of g_dispatch_scratch in that context
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
+
+// Driver calls resolved through the runtime (the library links no driver
+// library): the current context and its unique ID.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// ID of the context current on this thread, or 0 if there is none or the
+// driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {   // called with g_scratch_mutex held
+        cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f2);
+        resolved = true;
+    }
+    if (get_current == nullptr || get_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // The device address of the static scratch on the current device.  In host
 // code `g_dispatch_scratch` names a host-side stand-in, not device memory, so
-// the address must come from the runtime.
+// the address must come from the runtime: it is looked up once per device and
+// context, and again whenever the device's current context has changed.
 ep_status_t scratch_on_current_device(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -52,17 +94,21 @@ ep_status_t scratch_on_current_device(void** out) {
     }
     if (dev < 0 || dev >= kMaxDevices) return EP_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr& c = g_scratch[dev];
+    const unsigned long long id = current_context_id();
+    if (c.addr == nullptr || id == 0 || id != c.ctx_id) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
         if (e != cudaSuccess || p == nullptr) {
             fprintf(stderr, "libep: ep_dispatch_noalloc: cudaGetSymbolAddress failed on device %d (%s)\n", dev,
                     cudaGetErrorString(e));
+            c.addr = nullptr;
             return EP_ERR_CUDA;
         }
-        g_scratch_addr[dev] = p;
+        c.addr = p;
+        c.ctx_id = current_context_id();   // the lookup makes the device's context current if it was not
     }
-    *out = g_scratch_addr[dev];
+    *out = c.addr;
     return EP_OK;
 }
 

@@ -20,8 +20,6 @@
 //      kernel).  CTA 0 writes the per-expert / per-rank
 //      outputs and the status word.
 // No sort, no global atomics except the barrier counter.
-#include <stdlib.h>
-
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -119,9 +117,7 @@ __device__ int block_exclusive_scan_E(const int* in, int* out, int E, int* s_war
 }  // namespace
 
 template <int KT>
-// stall > 0 (a test of the bounded wait only) raises the first barrier's
-// target past the number of CTAs, so that no CTA can pass it.
-__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a, unsigned stall) {
+__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     grid_launch_dependents();   // the pack kernel may be scheduled; it waits for our results
     extern __shared__ int32_t smem[];
     const int E = a.E, K = KT > 0 ? KT : a.K, R = a.R, L = a.L;
@@ -239,7 +235,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a, unsigned s
         if (tid == 0) a.chunk_err[c] = *s_err;
         __syncthreads();
     }
-    if (!grid_barrier(a.barrier, (unsigned)G + stall, s_flag)) {
+    if (!grid_barrier(a.barrier, (unsigned)G + a.stall, s_flag)) {
         if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
         return;
     }
@@ -454,11 +450,7 @@ cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // EP_TEST_STALL_BARRIER=1 in the environment makes the first grid barrier
-    // unreachable, for tests of the timeout path (EP_ERR_TIMEOUT after 2 s)
-    const char* stall_env = getenv("EP_TEST_STALL_BARRIER");
-    const unsigned stall = stall_env != nullptr && stall_env[0] == '1' ? 1u : 0u;
-    return cudaLaunchKernelEx(&cfg, k_route<KT>, a, stall);
+    return cudaLaunchKernelEx(&cfg, k_route<KT>, a);
 }
 
 }  // namespace

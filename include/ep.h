@@ -26,9 +26,9 @@
  *     unspecified, but no kernel ever writes outside the buffers described
  *     here and none waits without a bound.
  *   - The routing kernel's grid barriers give up after 2 s (EP_ERR_TIMEOUT);
- *     the pack kernels of that call then write nothing.  For tests of that
- *     path, EP_TEST_STALL_BARRIER=1 in the environment makes the first
- *     barrier unreachable.
+ *     the pack kernels of that call then write nothing.  (ep_testing.h holds
+ *     test-only variants of the routing calls whose first barrier cannot be
+ *     reached; no environment variable or other state changes this path.)
  *   - Sizes: T tokens (all logical ranks together), K top-k entries per
  *     token, E experts, R logical ranks, L = E / R local experts per rank,
  *     H hidden channels, A expert alignment.  Token t belongs to source rank
@@ -232,7 +232,10 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* handle, const e
  * static device array of 2 MiB per GPU, held until the process exits; sizes
  * whose scratch (ep_workspace_bytes) exceeds 2 MiB return EP_ERR_INVALID_ARG
  * with a message on stderr, before anything runs.  The first call on a device
- * looks up the array's address (make it before any stream capture).  All
+ * looks up the array's address (make it before any stream capture); it is
+ * cached per device together with the ID of the current CUDA context, and a
+ * call in a new context of that device (after cudaDeviceReset) looks it up
+ * again, which should likewise precede any stream capture.  All
  * calls on a device share the array: calls whose kernels overlap on the GPU
  * race, so serialise them on one stream.  Allocates nothing.
  */

@@ -16,8 +16,8 @@ def lib():
     return C.CDLL(build.build())
 
 
-def declared_functions():
-    src = open(HEADER).read()
+def declared_functions(header=HEADER):
+    src = open(header).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ep_\w+)\s*\(", src, flags=re.M)
     return sorted(set(names))
@@ -34,6 +34,20 @@ def test_header_declares_the_calls():
 def test_every_declared_symbol_is_exported(lib):
     for n in declared_functions():
         assert hasattr(lib, n), n
+
+
+def test_testing_header_symbols_are_exported(lib):
+    names = declared_functions(os.path.join(ROOT, "include", "ep_testing.h"))
+    assert names == ["ep_testing_dispatch_stalled", "ep_testing_get_dispatch_layout_stalled"]
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_no_environment_switch_in_the_library():
+    # the bounded-wait tests reach the stalled routing through ep_testing.h only
+    for f in os.listdir(os.path.join(ROOT, "combine_topk_idx_rank_b200", "csrc")):
+        src = open(os.path.join(ROOT, "combine_topk_idx_rank_b200", "csrc", f)).read()
+        assert "getenv" not in src, f
 
 
 def test_binding_exports_match_header():

@@ -27,15 +27,18 @@ def test_algorithmic_bytes_worked_example():
     x_read = 4 * 16 * 2                  # every token row once
     rows_written = 10 * 16 * 2           # received rows, padding included
     per_row_meta = 10 * (2 * 2 * 4 + 8)  # recv_topk_idx + recv_topk_weights + recv_src_metadata
-    per_entry = 4 * 2 * (8 + 4 + 4)      # topk_idx + topk_weights read, dst_buffer_slot_idx written
-    assert ab["pack"] == x_read + rows_written + per_row_meta + per_entry
+    # routing: topk_idx + topk_weights read, the int32 id copy and dst_buffer_slot_idx written,
+    # the per-row metadata, psum and counts
+    assert ab["route"] == 4 * 2 * (8 + 4 + 4 + 4) + per_row_meta + 2 * 4 * 4
+    # pack: x once, dst_buffer_slot_idx read, every received row written
+    assert ab["pack"] == x_read + 4 * 2 * 4 + rows_written
     # combine: slots and weights read, each unmasked y row once, out once
     assert ab["combine"] == 4 * 2 * 8 + 8 * 16 * 2 + 4 * 16 * 2
     # FP8 group 8: one byte per element plus an fp32 scale per group; low-latency: no padding rows
     cfg8 = cfg.scaled(quant="fp8", quant_size=8)
     ab8 = bench.algorithmic_bytes(cfg8, [3, 0, 4, 1], 4, low_latency=True)
     assert ab8["rows_aligned"] == 8
-    assert ab8["pack"] == x_read + 8 * 16 + 8 * 2 * 4 + 8 * (2 * 2 * 4 + 8) + per_entry
+    assert ab8["pack"] == x_read + 4 * 2 * 4 + 8 * 16 + 8 * 2 * 4
     # quantised combine reads the codes and their scales instead of bf16 rows
     abq = bench.algorithmic_bytes(cfg8, [3, 0, 4, 1], 4, combine_quant=True)
     assert abq["combine"] == 4 * 2 * 8 + 8 * (16 + 2 * 4) + 4 * 16 * 2
@@ -51,6 +54,7 @@ def test_prefill_bytes_match_the_workload_counts():
     assert ab["rows_aligned"] == int((-(-counts // 128) * 128).sum())
     # x once (0.47 GB) + 8 bf16 copies (3.76 GB) + padding rows: about 4.5 GB
     assert 4.4e9 < ab["pack"] < 4.6e9 and 4.2e9 < ab["combine"] < 4.25e9
+    assert 0.02e9 < ab["route"] < 0.03e9
 
 
 def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):

@@ -85,3 +85,32 @@ def test_single_rank_helpers():
     assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
     assert bench.rank_seed(5, 3) == 8
     assert bench.job_tokens_per_s(1, 1000, 2.0) == pytest.approx(5e5)
+
+
+@pytest.mark.timeout(300)
+def test_launcher_starts_one_process_per_gpu():
+    """`bench.py --gpus 2` without a torchrun environment starts two ranks
+    itself; the reference arm then prints one JSON line (rank 0's) for a
+    two-GPU job and the other rank exits 0 without output."""
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "3", "--warmup", "3", "--ref-seconds", "2"],
+                       capture_output=True, text=True, env=env, timeout=280)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2 and rec["impl"] == "reference"
+    assert rec["config"]["name"] == "tiny" and rec["steps"] == 3
+    # the step time is measured: all steps fit in the run's own wall clock
+    assert rec["ms_per_step"] * rec["steps"] < 280e3
+
+
+def test_launch_ranks_reports_a_failing_rank(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    script = tmp_path / "fail_on_rank1.py"
+    script.write_text("import os, sys\nsys.exit(3 if os.environ['RANK'] == '1' else 0)\n")
+    monkeypatch.setattr(bench, "__file__", str(script))
+    assert bench.launch_ranks(2, [], timeout_s=60) == 3
