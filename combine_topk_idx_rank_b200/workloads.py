@@ -39,7 +39,7 @@ from typing import Dict, Optional
 
 import numpy as np
 
-__all__ = ["WorkloadConfig", "CONFIGS", "Workload", "make_workload", "make_y",
+__all__ = ["WorkloadConfig", "CONFIGS", "Workload", "make_workload", "make_y", "make_router_logits",
            "bf16_bits_from_f32", "bf16_bits_to_f32"]
 
 
@@ -161,3 +161,10 @@ def make_y(rows: int, hidden: int, seed: int, device: str = "cpu"):
     g = torch.Generator(device=device)
     g.manual_seed(seed + 0x5EED)
     return torch.randn((rows, hidden), generator=g, device=device, dtype=torch.bfloat16)
+
+
+def make_router_logits(tokens: int, experts: int, seed: int) -> np.ndarray:
+    """Router logits fp32 [tokens, experts] ~ N(0, 1) from PCG64 (seed + 0x6A7E),
+    the input of the group-limited gating generator."""
+    rng = np.random.default_rng(seed + 0x6A7E)
+    return rng.standard_normal((tokens, experts), dtype=np.float32)

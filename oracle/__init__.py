@@ -19,7 +19,7 @@ import numpy as np
 
 from . import build as _build
 
-OK, INVALID_ARG, BAD_EXPERT_ID, CAPACITY = 0, 1, 2, 3
+OK, INVALID_ARG, BAD_EXPERT_ID, CAPACITY, NONFINITE = 0, 1, 2, 3, 4
 QUANT = {"none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 
 
@@ -107,6 +107,8 @@ def _setup(L):
     L.oracle_f32_to_bf16_n.restype = None
     L.oracle_e4m3_to_f64_n.argtypes = [p, i64, p]
     L.oracle_e4m3_to_f64_n.restype = None
+    L.oracle_group_limited_gating.argtypes = [p, i32, i32, i32, i32, i32, p, p]
+    L.oracle_group_limited_gating.restype = C.c_int
     L.oracle_threads.argtypes = [C.c_int]
     L.oracle_threads.restype = C.c_int
     return L
@@ -397,3 +399,20 @@ def dispatch_rows_mx(x, dst_buffer_slot_idx, quant: str, quant_size: int, round_
     if st:
         raise OracleError(st, "dispatch_rows_mx")
     return recv_x, recv_scales
+
+
+# -------------------------------------------------- group-limited gating
+
+def group_limited_gating(logits, n_group: int, topk_group: int, per_group: int):
+    """(topk_idx int64 [T, K], topk_weights fp32 [T, K]) of group-limited
+    gating over router logits fp32 [T, E]: K = topk_group * per_group
+    (see ep_oracle.c for the definition and its readings)."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    K = topk_group * per_group
+    idx = np.zeros((T, K), np.int64)
+    w = np.zeros((T, K), np.float32)
+    st = lib().oracle_group_limited_gating(_ptr(lg), T, E, n_group, topk_group, per_group, _ptr(idx), _ptr(w))
+    if st:
+        raise OracleError(st, "group_limited_gating")
+    return idx, w

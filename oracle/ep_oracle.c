@@ -53,7 +53,7 @@
  * expert id of every top-k entry that lives on that rank, else -1.
  *
  * Status codes are this file's own (0 ok, 1 invalid argument, 2 expert id out
- * of range, 3 receive capacity too small).
+ * of range, 3 receive capacity too small, 4 a non-finite router logit).
  */
 #include <math.h>
 #include <stdint.h>
@@ -628,6 +628,96 @@ int oracle_dispatch_rows_mx(const uint16_t* x, int T, int H, int K, const int32_
         free(sc);
     }
     return st;
+}
+
+/* ---------------------------------------------- group-limited gating */
+
+#define OR_NONFINITE 4
+
+/* Group-limited gating, the routing that produces topk_idx / topk_weights
+ * upstream of dispatch ("DeepEP V1 vs V2 comparative analysis", section 8.1,
+ * DeepSeek-V3 group-limited gating: 256 experts in 32 groups of 8, each token
+ * keeps its top-4 groups, then the top-2 experts inside each kept group, top-8
+ * experts in all).  logits: fp32 [T, E]; the E experts form n_group groups of
+ * E / n_group consecutive ids; K = topk_group * per_group entries per token.
+ *
+ * Readings where the page is silent (one each):
+ *  - an expert's affinity is its router logit; of two experts the one with
+ *    the larger logit ranks first, and of two equal logits the lower id;
+ *  - a group's score is the fp32 sum of its per_group largest logits, added
+ *    from the largest down (so the kept groups are those whose picks add up
+ *    highest); of two equal scores the lower group id ranks first;
+ *  - the K entries of a token are listed by logit, largest first, equal
+ *    logits by lower id;
+ *  - topk_weights[t] is the softmax over the K selected logits, computed in
+ *    binary64 and rounded to binary32.
+ * Logits must be finite: a NaN or infinite logit returns OR_NONFINITE.
+ * Steps, in the page's order: per group its best experts and score; the
+ * topk_group best groups; the per_group best experts of each kept group;
+ * order and weights. */
+int oracle_group_limited_gating(const float* logits, int T, int E, int n_group, int topk_group, int per_group,
+                                int64_t* topk_idx, float* topk_weights) {
+    if (T < 0 || E < 1 || n_group < 1 || E % n_group != 0) return OR_INVALID_ARG;
+    const int S = E / n_group;
+    if (topk_group < 1 || topk_group > n_group || per_group < 1 || per_group > S) return OR_INVALID_ARG;
+    const int K = topk_group * per_group;
+    int* pick = malloc(sizeof(int) * (size_t)E);         /* [n_group][per_group] best experts per group */
+    float* score = malloc(sizeof(float) * (size_t)n_group);
+    char* taken = malloc((size_t)(E > n_group ? E : n_group));
+    int* sel = malloc(sizeof(int) * (size_t)K);
+    int status = OR_OK;
+    for (int t = 0; t < T && status == OR_OK; ++t) {
+        const float* l = logits + (int64_t)t * E;
+        for (int e = 0; e < E; ++e)
+            if (!isfinite(l[e])) status = OR_NONFINITE;
+        if (status) break;
+        /* 1. every group's per_group best experts, and its score */
+        memset(taken, 0, (size_t)E);
+        for (int g = 0; g < n_group; ++g) {
+            for (int j = 0; j < per_group; ++j) {
+                int best = -1;
+                for (int e = g * S; e < (g + 1) * S; ++e)
+                    if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+                taken[best] = 1;
+                pick[g * per_group + j] = best;
+            }
+            float sc = l[pick[g * per_group]];
+            for (int j = 1; j < per_group; ++j) sc = sc + l[pick[g * per_group + j]];
+            score[g] = sc;
+        }
+        /* 2. the topk_group best groups; 3. their picks */
+        memset(taken, 0, (size_t)n_group);
+        int n = 0;
+        for (int j = 0; j < topk_group; ++j) {
+            int best = -1;
+            for (int g = 0; g < n_group; ++g)
+                if (!taken[g] && (best < 0 || score[g] > score[best])) best = g;
+            taken[best] = 1;
+            for (int i = 0; i < per_group; ++i) sel[n++] = pick[best * per_group + i];
+        }
+        /* 4. order: larger logit first, equal logits by lower id (insertion sort) */
+        for (int i = 1; i < K; ++i) {
+            int v = sel[i], j = i - 1;
+            while (j >= 0 && (l[sel[j]] < l[v] || (l[sel[j]] == l[v] && sel[j] > v))) {
+                sel[j + 1] = sel[j];
+                --j;
+            }
+            sel[j + 1] = v;
+        }
+        /* 5. softmax over the K selected logits in binary64, rounded to binary32 */
+        const double m = (double)l[sel[0]];
+        double sum = 0.0;
+        for (int k = 0; k < K; ++k) sum += exp((double)l[sel[k]] - m);
+        for (int k = 0; k < K; ++k) {
+            topk_idx[(int64_t)t * K + k] = sel[k];
+            topk_weights[(int64_t)t * K + k] = (float)(exp((double)l[sel[k]] - m) / sum);
+        }
+    }
+    free(pick);
+    free(score);
+    free(taken);
+    free(sel);
+    return status;
 }
 
 /* ------------------------------------------------------------- threads */

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__)
 sys.path.insert(0, ROOT)
 
 import oracle  # noqa: E402
-from combine_topk_idx_rank_b200.workloads import CONFIGS, make_workload, make_y  # noqa: E402
+from combine_topk_idx_rank_b200.workloads import CONFIGS, make_router_logits, make_workload, make_y  # noqa: E402
 
 OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_digests.json")
 
@@ -57,6 +57,11 @@ def compute():
             entry["num_recv_rows"] = int(d["num_recv_rows"])
             entry["combined"] = digest(out)
             res[f"{name}/seed{seed}"] = entry
+    # group-limited gating at the DeepSeek-V3 shape (256 experts, 32 groups,
+    # top-4 groups, top-2 per group) on 512 tokens of seeded router logits
+    for seed in (0, 1, 2):
+        idx, w = oracle.group_limited_gating(make_router_logits(512, 256, seed), 32, 4, 2)
+        res[f"gating_dsv3_512/seed{seed}"] = {"topk_idx": digest(idx), "topk_weights": digest(w)}
     return res
 
 
