@@ -37,7 +37,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from combine_topk_idx_rank_b200.workloads import CONFIGS, make_workload  # noqa: E402
+from combine_topk_idx_rank_b200.workloads import CONFIGS, make_router_logits, make_workload  # noqa: E402
 
 METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) on 1 B200"
 UNIT = "tokens/s"
@@ -250,7 +250,7 @@ def barrier(world: int):
 def config_dict(args, cfg, world):
     """The `config` object of the JSON line; both arms print the same one."""
     T, H, K, E, R = cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks
-    opt = {"mode": "full", "tokens": 0, "quant": None, "ue8m0": False, "combine_quant": False}
+    opt = {"mode": "full", "tokens": 0, "quant": None, "ue8m0": False, "combine_quant": False, "gating": False}
     opt.update({k: getattr(args, k) for k in opt if hasattr(args, k)})
     args = argparse.Namespace(workload=args.workload, **opt)
     ll = args.mode == "ll"
@@ -262,7 +262,9 @@ def config_dict(args, cfg, world):
             + (" — low-latency fixed-capacity layout" if ll else "")
             + (f" — dispatch {cfg.quant} g{cfg.quant_size}{' ue8m0 bytes' if args.ue8m0 else ''}"
                if args.quant or args.ue8m0 else "")
-            + (" — combine reads the quantised rows" if args.combine_quant else ""),
+            + (" — combine reads the quantised rows" if args.combine_quant else "")
+            + (" — routing by group-limited gating (32 groups, top-4 groups, top-2 each) of N(0,1) router "
+               "logits, timed in the step" if args.gating else ""),
             "name": args.workload, "mode": args.mode, "tokens": T, "hidden": H,
             "num_experts": E, "num_ranks": R, "topk": K, "expert_alignment": cfg.expert_alignment,
             "quant": cfg.quant, "num_rounds": cfg.num_rounds,
@@ -305,6 +307,13 @@ def run_ours(args):
                    "recv_topk_weights": bufs.recv_topk_weights,
                    "count": torch.empty((E,), dtype=torch.int32, device=dev),
                    "layout_range": torch.empty((E, R), dtype=torch.int64, device=dev), "handle": bufs.handle}
+    if args.gating:
+        # the step starts from router logits: group-limited gating produces the routing
+        if E % 32 or K != 8 or args.mode != "full":
+            raise SystemExit("--gating needs 256-style experts in 32 groups, top-8, and --mode full")
+        logits = torch.from_numpy(make_router_logits(T, E, rank_seed(args.seed, rank))).to(dev)
+        gerr = torch.zeros((1,), dtype=torch.int32, device=dev)
+        ep.ep_group_limited_gating(logits, 32, 4, 2, out=(ti, tw), err=gerr)
     cap = bufs.recv_x.shape[0]
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     if args.combine_quant:
@@ -319,10 +328,13 @@ def run_ours(args):
                        quant_size=cfg.quant_size, round_scale=cfg.round_scale, num_rounds=cfg.num_rounds,
                        do_cpu_sync=False, buffers=bufs)
 
-    def step(evs=None, x=x, ti=ti, tw=tw, out=out):
-        """One dispatch + combine.  evs = four recorded events for the
-        per-kernel split (step start, pack begin, pack end, combine end), or
-        None: then nothing is recorded between the kernels."""
+    def step(evs=None, x=x, ti=ti, tw=tw, out=out, lg=None):
+        """One dispatch + combine (preceded by gating with --gating).  evs =
+        four recorded events for the per-kernel split (step start, pack begin,
+        pack end, combine end), or None: then nothing is recorded between the
+        kernels."""
+        if args.gating:
+            ep.ep_group_limited_gating(logits if lg is None else lg, 32, 4, 2, out=(ti, tw), err=gerr, check=False)
         if evs is not None:
             evs[0].record()
         pev = None if evs is None else (evs[1], evs[2])
@@ -353,6 +365,8 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     bufs.handle.check()
+    if args.gating:
+        assert int(gerr.item()) == 0
     counts = bufs.handle.num_recv_tokens_per_expert.cpu().numpy()
 
     # ------------------------------------------------- headline timed region
@@ -395,6 +409,7 @@ def run_ours(args):
     hx = torch.from_numpy(wl.x.view(np.int16)).view(torch.bfloat16).pin_memory()
     hti = torch.from_numpy(wl.topk_idx).pin_memory()
     htw = torch.from_numpy(wl.topk_weights).pin_memory()
+    hlg = logits.cpu().pin_memory() if args.gating else None
     hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
 
     # two device input / output sets: step i's host->device copies run on one
@@ -406,6 +421,7 @@ def run_ours(args):
     dx = [torch.empty_like(x) for _ in range(2)]
     dti = [torch.empty_like(ti) for _ in range(2)]
     dtw = [torch.empty_like(tw) for _ in range(2)]
+    dlg = [torch.empty_like(logits) for _ in range(2)] if args.gating else [None, None]
     dout = [torch.empty_like(out) for _ in range(2)]
     hout2 = [hout, torch.empty_like(hout).pin_memory()]
     ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -419,12 +435,15 @@ def run_ours(args):
         s_in.wait_event(ev_done[b])              # step i-2 has finished reading set b
         with torch.cuda.stream(s_in):
             dx[b].copy_(hx, non_blocking=True)
-            dti[b].copy_(hti, non_blocking=True)
-            dtw[b].copy_(htw, non_blocking=True)
+            if args.gating:                  # the routing is computed on the device from the logits
+                dlg[b].copy_(hlg, non_blocking=True)
+            else:
+                dti[b].copy_(hti, non_blocking=True)
+                dtw[b].copy_(htw, non_blocking=True)
             ev_in[b].record(s_in)
         comp.wait_event(ev_in[b])
         comp.wait_event(ev_free[b])              # step i-2's result has left dout[b]
-        step(None, dx[b], dti[b], dtw[b], dout[b])
+        step(None, dx[b], dti[b], dtw[b], dout[b], dlg[b])
         ev_done[b].record(comp)
         s_out.wait_event(ev_done[b])
         with torch.cuda.stream(s_out):
@@ -447,14 +466,15 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     assert torch.equal(hout2[(e2e_steps - 1) % 2].view(torch.int16), out.cpu().view(torch.int16))
-    h2d = hx.numel() * 2 + hti.numel() * 8 + htw.numel() * 4
+    h2d = hx.numel() * 2 + (hlg.numel() * 4 if args.gating else hti.numel() * 8 + htw.numel() * 4)
     d2h = hout.numel() * 2
 
     ab = algorithmic_bytes(cfg, counts, T, ue8, args.combine_quant, ll)
     if args.mode == "cached":
         ab["route"] = 0
+    ab["gating"] = T * E * 4 + T * K * 12 if args.gating else 0     # logits read, ids and weights written
     ms_per_step = elapsed_ms / args.steps
-    step_bytes = ab["route"] + ab["pack"] + ab["combine"]
+    step_bytes = ab["gating"] + ab["route"] + ab["pack"] + ab["combine"]
     value = job_tokens_per_s(world, T, ms_per_step)
     gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
@@ -467,9 +487,9 @@ def run_ours(args):
                                            combine_ms / cfg.num_rounds)
     clocks = sampler.summary(t_wall0, t_wall1)
     default_launch = (args.mode == "full" and not args.quant and not args.ue8m0 and not args.combine_quant
-                      and not args.tokens)
+                      and not args.tokens and not args.gating)
     # routing (1 cooperative kernel) unless cached, pack x rounds, combine x rounds
-    launches_per_step = (0 if args.mode == "cached" else 1) + 2 * cfg.num_rounds
+    launches_per_step = (0 if args.mode == "cached" else 1) + 2 * cfg.num_rounds + (1 if args.gating else 0)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -480,7 +500,8 @@ def run_ours(args):
         "hbm": {"achieved_gbs": round(gbs, 1), "algorithmic_bytes_per_step": step_bytes,
                 "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "frac_of_measured": round(gbs / peak, 4),
                 "measured_peak_gbs": peak, "rows": ab["rows"], "rows_aligned": ab["rows_aligned"],
-                "bytes": {"route": ab["route"], "pack": ab["pack"], "combine": ab["combine"]}},
+                "bytes": {"gating": ab["gating"], "route": ab["route"], "pack": ab["pack"],
+                          "combine": ab["combine"]}},
         "kernels": {"route_ms": round(route_ms, 5), "pack_ms": round(pack_ms, 5), "pack_gbs": round(pack_gbs, 1),
                     "combine_ms": round(combine_ms, 5), "combine_gbs": round(combine_gbs, 1),
                     "split_steps": n_split, "split_step_ms": round(split_step_ms, 5),
@@ -500,7 +521,8 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, wl, step_bytes / T, budget_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(cfg, wl, step_bytes / T, budget_s=args.cpu_seconds,
+                                              logits=logits.cpu().numpy() if args.gating else None)
     if rank == 0:
         print(json.dumps(result), flush=True)
     barrier(world)
@@ -526,9 +548,10 @@ class OracleSampler:
 
     POOL = 8192
 
-    def __init__(self, cfg, wl, seed=0):
+    def __init__(self, cfg, wl, seed=0, logits=None):
         from combine_topk_idx_rank_b200.workloads import make_y
         self.cfg, self.wl = cfg, wl
+        self.logits = logits            # router logits: the routing comes from group-limited gating
         self.ypool = make_y(self.POOL, cfg.hidden, 7)
         self.rng = np.random.default_rng(seed)
 
@@ -545,7 +568,10 @@ class OracleSampler:
         import oracle
         cfg, wl = self.cfg, self.wl
         idx, w, x = wl.topk_idx[tok], wl.topk_weights[tok], wl.x[tok]
+        lg = None if self.logits is None else self.logits[tok]
         t0 = time.perf_counter()
+        if lg is not None:
+            idx, w = oracle.group_limited_gating(lg, 32, 4, 2)
         s = oracle.slots(idx, w, cfg.num_experts, cfg.num_ranks, cfg.expert_alignment)
         dst = s["dst_buffer_slot_idx"]
         pdst = np.where(dst >= 0, dst % self.POOL, -1).astype(np.int32)
@@ -560,12 +586,12 @@ class OracleSampler:
         return self.run(tok) / tok.size
 
 
-def cpu_baseline(cfg, wl, bytes_per_token, budget_s=12.0):
+def cpu_baseline(cfg, wl, bytes_per_token, budget_s=12.0, logits=None):
     """The oracle timed on this host's cores: the single-threaded build on one
     core, then the OpenMP build of the same source on every core in
     sched_getaffinity, each on measured token samples (no projection)."""
     import oracle
-    smp = OracleSampler(cfg, wl)
+    smp = OracleSampler(cfg, wl, logits=logits)
     res = {}
     for label, n in (("one_core", 1), ("all_cores", host_cores())):
         used = oracle.use_threads(n)
@@ -599,7 +625,8 @@ def run_reference(args):
     T = cfg.num_tokens
     cores = host_cores()
     used = oracle.use_threads(cores)
-    smp = OracleSampler(cfg, wl, seed=args.seed)
+    logits = make_router_logits(T, cfg.num_experts, args.seed) if getattr(args, "gating", False) else None
+    smp = OracleSampler(cfg, wl, seed=args.seed, logits=logits)
     per_tok = smp.calibrate()
     n_steps = args.steps + args.warmup
     per_rank = int(max(1, (args.ref_seconds / n_steps) / per_tok / cfg.num_ranks))
@@ -684,6 +711,8 @@ def main(argv=None):
     p.add_argument("--ue8m0", action="store_true", help="power-of-two scales stored as UE8M0 bytes")
     p.add_argument("--combine-quant", action="store_true",
                    help="combine reads the FP8 / int8 received rows (identity experts) instead of bf16 y")
+    p.add_argument("--gating", action="store_true",
+                   help="each step starts from router logits: group-limited gating, then dispatch and combine")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the cpu_baseline samples")
     p.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the --impl reference run")
     p.add_argument("--no-cpu-baseline", action="store_true")

@@ -7,7 +7,7 @@ on first use, so importing the input generators (``workloads``) does not need
 the CUDA library.
 """
 
-_API = ("ep_get_dispatch_layout", "ep_dispatch", "ep_combine", "EPHandle",
+_API = ("ep_get_dispatch_layout", "ep_dispatch", "ep_combine", "ep_group_limited_gating", "EPHandle",
         "DispatchBuffers", "alloc_dispatch_buffers", "EPError", "recv_capacity_bound",
         "workspace_bytes", "library_path")
 

@@ -136,6 +136,7 @@ const char* ep_status_string(ep_status_t s) {
         case EP_ERR_CAPACITY: return "receive capacity too small";
         case EP_ERR_CUDA: return "CUDA error";
         case EP_ERR_TIMEOUT: return "device wait timed out";
+        case EP_ERR_NONFINITE: return "router logit not finite";
     }
     return "unknown status";
 }
@@ -385,6 +386,24 @@ ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant,
 ep_status_t ep_combine(const void* y, const ep_handle_t* h, const float* topk_weights, void* out,
                        void* stream) {
     return ep_combine_ex(y, nullptr, EP_QUANT_NONE, 0, h, topk_weights, nullptr, out, stream);
+}
+
+ep_status_t ep_group_limited_gating(const float* logits, int32_t T, int32_t E, int32_t n_group,
+                                    int32_t topk_group, int32_t per_group, int64_t* topk_idx,
+                                    float* topk_weights, int32_t* err, void* stream) {
+    if (T < 0 || T > (1 << 24) || E < 1 || E > kMaxExperts) return EP_ERR_INVALID_ARG;
+    if (n_group < 1 || n_group > 32 || E % n_group != 0) return EP_ERR_INVALID_ARG;
+    if (topk_group < 1 || topk_group > n_group || per_group < 1 || per_group > E / n_group) return EP_ERR_INVALID_ARG;
+    if (topk_group * per_group > kMaxTopk) return EP_ERR_INVALID_ARG;
+    if (err == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (logits == nullptr || topk_idx == nullptr || topk_weights == nullptr)) return EP_ERR_INVALID_ARG;
+    GateArgs g{};
+    g.logits = logits;
+    g.T = T; g.E = E; g.n_group = n_group; g.topk_group = topk_group; g.per_group = per_group;
+    g.vec_ok = aligned16(logits) && E % 4 == 0;
+    g.topk_idx = topk_idx; g.topk_weights = topk_weights;
+    g.err = err;
+    return cuda_status(launch_gate(g, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status) {

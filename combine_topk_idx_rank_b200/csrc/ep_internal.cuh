@@ -135,10 +135,21 @@ struct CombineArgs {
     int32_t* err;
 };
 
+struct GateArgs {
+    const float* logits;        // [T, E] router logits
+    int64_t T;
+    int E, n_group, topk_group, per_group;
+    int vec_ok;                 // logits 16-byte aligned (rows of E % 4 == 0 floats)
+    int64_t* topk_idx;          // [T, K]
+    float* topk_weights;        // [T, K]
+    int32_t* err;               // [1] status word (cleared by the launch)
+};
+
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+cudaError_t launch_gate(const GateArgs& a, cudaStream_t st);
 
 int device_sm_count();
 

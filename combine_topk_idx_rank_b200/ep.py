@@ -29,12 +29,13 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(HERE, "libep.so")
 
-EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, EP_ERR_TIMEOUT = range(6)
+(EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_EXPERT_ID, EP_ERR_CAPACITY, EP_ERR_CUDA, EP_ERR_TIMEOUT,
+ EP_ERR_NONFINITE) = range(7)
 _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
-            "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex")
+            "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex", "ep_group_limited_gating")
 
 
 class EPError(RuntimeError):
@@ -87,6 +88,8 @@ def _load(path: str = _LIB_PATH):
     L.ep_read_error.restype = C.c_int
     L.ep_copy_recv_counts.argtypes = [C.POINTER(_Handle), p, p, C.POINTER(C.c_int64)]
     L.ep_copy_recv_counts.restype = C.c_int
+    L.ep_group_limited_gating.argtypes = [p, i32, i32, i32, i32, i32, p, p, p, p]
+    L.ep_group_limited_gating.restype = C.c_int
     L.ep_status_string.argtypes = [C.c_int]
     L.ep_status_string.restype = C.c_char_p
     return L
@@ -470,3 +473,36 @@ def ep_dispatch_low_latency(x: torch.Tensor, topk_idx: torch.Tensor, topk_weight
     rs = b["recv_scales"]
     return (b["recv_x"].view(E, R * M, -1), None if rs is None else rs.view(E, R * M, -1), b["count"],
             b["layout_range"], h)
+
+
+@_on_tensor_device
+def ep_group_limited_gating(logits: torch.Tensor, n_group: int = 32, topk_group: int = 4, per_group: int = 2, *,
+                            out: Optional[tuple] = None, err: Optional[torch.Tensor] = None, check: bool = True):
+    """Group-limited gating (DeepSeek-V3): router logits fp32 [T, E] ->
+    (topk_idx int64 [T, K], topk_weights fp32 [T, K]), K = topk_group * per_group,
+    ready for ep_dispatch.  The defaults are the DeepSeek-V3 setting (32 groups,
+    top-4 groups, top-2 experts per group).  ``out`` = (topk_idx, topk_weights)
+    preallocated; ``err`` an int32 [1] status word; with ``check`` the call
+    waits and raises on a device error (EP_ERR_NONFINITE)."""
+    _need_cuda(logits, "logits", torch.float32)
+    T, E = logits.shape
+    K = topk_group * per_group
+    dev = logits.device
+    if out is None:
+        out = (torch.empty((T, K), dtype=torch.int64, device=dev), torch.empty((T, K), dtype=torch.float32, device=dev))
+    idx, w = out
+    _need_cuda(idx, "topk_idx", torch.int64)
+    _need_cuda(w, "topk_weights", torch.float32)
+    if tuple(idx.shape) != (T, K) or tuple(w.shape) != (T, K):
+        raise ValueError("out tensors must be [T, topk_group * per_group]")
+    if err is None:
+        err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    st = _lib.ep_group_limited_gating(_ptr(logits), T, E, n_group, topk_group, per_group, _ptr(idx), _ptr(w),
+                                      _ptr(err), _stream(dev))
+    _check(st, "ep_group_limited_gating")
+    if check:
+        s = C.c_int32(0)
+        _check(_lib.ep_read_error(_ptr(err), _stream(dev), C.byref(s)), "ep_read_error")
+        if s.value:
+            raise EPError(s.value, "ep_group_limited_gating")
+    return idx, w

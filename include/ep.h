@@ -53,8 +53,9 @@ typedef enum {
     EP_ERR_BAD_EXPERT_ID = 2, /* some topk_idx entry is < -1 or >= E (device) */
     EP_ERR_CAPACITY = 3,      /* recv_capacity < rows needed (device) */
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed */
-    EP_ERR_TIMEOUT = 5        /* a bounded device wait gave up (routing's grid barrier
+    EP_ERR_TIMEOUT = 5,       /* a bounded device wait gave up (routing's grid barrier
                                  waits at most 2 s); nothing is packed after it */
+    EP_ERR_NONFINITE = 6      /* a router logit is NaN or infinite (gating, device) */
 } ep_status_t;
 
 typedef enum {
@@ -278,6 +279,34 @@ ep_status_t ep_combine(const void* y, const ep_handle_t* handle, const float* to
 ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,
                           const ep_handle_t* handle, const float* topk_weights, const void* shared, void* out,
                           void* stream);
+
+/*
+ * Group-limited gating: the routing generator whose topk_idx / topk_weights
+ * feed ep_dispatch ("DeepEP V1 vs V2 comparative analysis", section 8.1,
+ * DeepSeek-V3 group-limited gating: 256 experts in 32 groups of 8, each token
+ * keeps its top-4 groups and the top-2 experts inside each, top-8 in all).
+ * For every token t of router logits [T, E]:
+ *   - the experts form n_group groups of E / n_group consecutive ids;
+ *   - a group's score is the fp32 sum of its per_group largest logits, added
+ *     from the largest down;
+ *   - the topk_group best groups are kept, and the per_group best experts of
+ *     each are the token's K = topk_group * per_group entries, listed by
+ *     logit, largest first;
+ *   - of two equal logits or scores, the lower expert / group id ranks first;
+ *   - topk_weights[t] = softmax over the K selected logits, computed in
+ *     binary64 and rounded to binary32.
+ *   logits         device fp32 [T, E]
+ *   topk_idx       device int64 [T, K] (output; K distinct ids in [0, E))
+ *   topk_weights   device fp32 [T, K] (output)
+ *   err            device int32 [1]: status word, cleared by this call;
+ *                  EP_ERR_NONFINITE if a logit is NaN or infinite (the outputs
+ *                  are then unspecified but still K distinct ids in range)
+ * Limits: 0 <= T <= 2^24, 1 <= n_group <= 32, E % n_group == 0, E <= 1024,
+ * 1 <= topk_group <= n_group, 1 <= per_group <= E / n_group, K <= 16.
+ */
+ep_status_t ep_group_limited_gating(const float* logits, int32_t T, int32_t E, int32_t n_group,
+                                    int32_t topk_group, int32_t per_group, int64_t* topk_idx,
+                                    float* topk_weights, int32_t* err, void* stream);
 
 /* Waits for `stream`, then copies the device status word to *host_status.
  * Returns EP_OK, or EP_ERR_CUDA if the wait or the copy failed. */
