@@ -65,7 +65,7 @@ RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const
 // and unaligned counts.
 ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R, int quant, int quant_size,
                                const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
-                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st) {
+                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st, bool after_routing) {
     ep_status_t s;
     if (opts->event_pack_begin) {
         s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
@@ -87,6 +87,12 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
+            pa.staged = 1;
+            pa.scales16 = aligned16(recv_scales);
+            // x was written before this call's routing kernel started, so the
+            // pack may read it while routing runs; a cached dispatch has no
+            // routing kernel before it and waits for its predecessor first
+            pa.prefetch = after_routing ? 1 : 0;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }
@@ -219,10 +225,11 @@ ep_status_t dispatch_impl(const void* x, int32_t T, int32_t H, const int64_t* to
     r.cumulative = opts->cumulative_local_expert_recv_stats;
     r.err_out = h->err;
     r.stall = stall;
+    r.token_offset = opts->token_offset;
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, recv_capacity, h,
-                              st);
+                              st, true);
 }
 
 }  // namespace
@@ -320,9 +327,10 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
     r.num_tokens_per_expert = packed_recv_count;
     r.cumulative = opts->cumulative_local_expert_recv_stats;
     r.err_out = h->err;
+    r.token_offset = opts->token_offset;
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st);
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st, true);
 }
 
 ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dispatch_opts_t* opts,
@@ -344,7 +352,7 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
     if (h->recv_capacity > 0 && recv_x == nullptr) return EP_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, h->recv_capacity, h,
-                              static_cast<cudaStream_t>(stream));
+                              static_cast<cudaStream_t>(stream), false);
 }
 
 ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,
@@ -404,6 +412,24 @@ ep_status_t ep_group_limited_gating(const float* logits, int32_t T, int32_t E, i
     g.topk_idx = topk_idx; g.topk_weights = topk_weights;
     g.err = err;
     return cuda_status(launch_gate(g, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_write_padding_rows(const int32_t* psum, const int32_t* counts, int32_t n_experts, void* recv_x,
+                                  int64_t row_bytes, void* recv_scales, int64_t scale_row_bytes,
+                                  int32_t* recv_topk_idx, float* recv_topk_weights, int32_t K,
+                                  int32_t* recv_src_metadata, int64_t capacity, void* stream) {
+    if (n_experts < 1 || n_experts > kMaxExperts || psum == nullptr || counts == nullptr) return EP_ERR_INVALID_ARG;
+    if (capacity < 0 || row_bytes < 16 || row_bytes % 16 != 0 || scale_row_bytes < 0) return EP_ERR_INVALID_ARG;
+    if (K < 1 || K > kMaxTopk) return EP_ERR_INVALID_ARG;
+    if (capacity > 0 && (recv_x == nullptr || !aligned16(recv_x))) return EP_ERR_INVALID_ARG;
+    if (capacity == 0) return EP_OK;
+    PadArgs p{};
+    p.psum = psum; p.cnt = counts; p.n = n_experts;
+    p.recv_x = static_cast<uint8_t*>(recv_x); p.row_bytes = row_bytes;
+    p.recv_scales = static_cast<uint8_t*>(recv_scales); p.scale_row_bytes = recv_scales ? scale_row_bytes : 0;
+    p.recv_topk_idx = recv_topk_idx; p.recv_topk_weights = recv_topk_weights; p.K = K;
+    p.recv_meta = recv_src_metadata; p.capacity = capacity;
+    return cuda_status(launch_padding(p, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status) {

@@ -75,6 +75,7 @@ struct RouteArgs {
     int T, K, E, R, L, A, log2_chunk, nchunks;
     int tokens_per_rank, chunks_per_rank;
     int ll_M;                   // > 0: low-latency layout with this many rows per (expert, source rank)
+    int token_offset;           // added to the token index written to recv_src_metadata
     int64_t* layout_range;      // [E,R] (low-latency layout) or null
     int64_t capacity;
     int check_capacity;
@@ -118,6 +119,10 @@ struct PackArgs {
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
     int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
+    int staged;                 // group quantisation may stage rows in shared memory
+    int scales16;               // recv_scales is 16-byte aligned (bulk stores of scale rows)
+    int prefetch;               // x may be read before the routing kernel has finished (the pack
+                                // follows this call's routing, which started after x was written)
     int32_t* err;
 };
 
@@ -145,11 +150,27 @@ struct GateArgs {
     int32_t* err;               // [1] status word (cleared by the launch)
 };
 
+struct PadArgs {
+    const int32_t* psum;        // [n] inclusive prefix of the aligned counts
+    const int32_t* cnt;         // [n] unaligned counts
+    int n;
+    uint8_t* recv_x;
+    int64_t row_bytes;
+    uint8_t* recv_scales;       // or null
+    int64_t scale_row_bytes;
+    int32_t* recv_topk_idx;     // [cap, K] or null
+    float* recv_topk_weights;   // [cap, K] or null
+    int K;
+    int32_t* recv_meta;         // [cap, 2] or null
+    int64_t capacity;
+};
+
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t st);
+cudaError_t launch_padding(const PadArgs& a, cudaStream_t st);
 
 int device_sm_count();
 

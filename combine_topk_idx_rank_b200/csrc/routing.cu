@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             }
             a.dst_slot[e0 + i] = slot;
             if (slot < 0) continue;
-            reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(t0 + tl, k);
+            reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(a.token_offset + t0 + tl, k);
             const int rdst = rank_of(e, L, shL);
             const int lo = rdst * L;   // local ids of the receiving rank: [lo, lo + L)
             const int* ids = s_idx + tl * K;

@@ -35,7 +35,8 @@ _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
-            "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex", "ep_group_limited_gating")
+            "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex", "ep_group_limited_gating",
+            "ep_write_padding_rows")
 
 
 class EPError(RuntimeError):
@@ -48,7 +49,7 @@ class _Opts(C.Structure):
     _fields_ = [("expert_alignment", C.c_int32), ("quant", C.c_int32), ("quant_size", C.c_int32),
                 ("round_scale", C.c_int32), ("num_rounds", C.c_int32), ("scale_ue8m0", C.c_int32),
                 ("cumulative_local_expert_recv_stats", C.c_void_p),
-                ("event_pack_begin", C.c_void_p), ("event_pack_end", C.c_void_p)]
+                ("event_pack_begin", C.c_void_p), ("event_pack_end", C.c_void_p), ("token_offset", C.c_int32)]
 
 
 class _Handle(C.Structure):
@@ -90,6 +91,8 @@ def _load(path: str = _LIB_PATH):
     L.ep_copy_recv_counts.restype = C.c_int
     L.ep_group_limited_gating.argtypes = [p, i32, i32, i32, i32, i32, p, p, p, p]
     L.ep_group_limited_gating.restype = C.c_int
+    L.ep_write_padding_rows.argtypes = [p, p, i32, p, i64, p, i64, p, p, i32, p, i64, p]
+    L.ep_write_padding_rows.restype = C.c_int
     L.ep_status_string.argtypes = [C.c_int]
     L.ep_status_string.restype = C.c_char_p
     return L
@@ -306,8 +309,11 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
                 recv_capacity: Optional[int] = None, buffers: Optional[DispatchBuffers] = None,
                 cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
                 layout_out: Optional[tuple] = None, events: Optional[tuple] = None,
-                handle: Optional[EPHandle] = None, scale_ue8m0: bool = False):
+                handle: Optional[EPHandle] = None, scale_ue8m0: bool = False, token_offset: int = 0):
     """Dispatch: returns (recv_x, recv_scales, recv_topk_idx, recv_topk_weights, handle).
+
+    ``token_offset`` is added to the token index of recv_src_metadata (tokens
+    [o, o + T) of a batch that spans several GPUs).
 
     With ``do_cpu_sync`` the call waits for the GPU, checks the status word and
     trims the outputs to the rows received (``handle.num_recv_rows``); without
@@ -347,7 +353,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor] = None,
                  None if cumulative_local_expert_recv_stats is None
                  else cumulative_local_expert_recv_stats.data_ptr(),
                  None if events is None else events[0].cuda_event,
-                 None if events is None else events[1].cuda_event)
+                 None if events is None else events[1].cuda_event, int(token_offset))
     ch = h._c()
     lay = layout_out or (None, None, None)
     stream = _stream(x.device)
@@ -506,3 +512,24 @@ def ep_group_limited_gating(logits: torch.Tensor, n_group: int = 32, topk_group:
         if s.value:
             raise EPError(s.value, "ep_group_limited_gating")
     return idx, w
+
+
+@_on_tensor_device
+def ep_write_padding_rows(psum: torch.Tensor, counts: torch.Tensor, recv_x: torch.Tensor,
+                          recv_scales: Optional[torch.Tensor] = None, recv_topk_idx: Optional[torch.Tensor] = None,
+                          recv_topk_weights: Optional[torch.Tensor] = None,
+                          recv_src_metadata: Optional[torch.Tensor] = None):
+    """Writes the alignment padding rows of a receive layout (psum / counts per
+    expert segment) as ep_dispatch writes them: zero rows and scales,
+    recv_topk_idx -1, weight 0, metadata (-1, -1)."""
+    _need_cuda(psum, "psum", torch.int32)
+    _need_cuda(counts, "counts", torch.int32)
+    _need_cuda(recv_x, "recv_x")
+    cap = recv_x.shape[0]
+    row_bytes = recv_x[0].numel() * recv_x.element_size() if cap else 16
+    srb = 0 if recv_scales is None else recv_scales[0].numel() * recv_scales.element_size()
+    K = recv_topk_idx.shape[1] if recv_topk_idx is not None else 1
+    st = _lib.ep_write_padding_rows(_ptr(psum), _ptr(counts), psum.numel(), _ptr(recv_x), row_bytes,
+                                    _ptr(recv_scales), srb, _ptr(recv_topk_idx), _ptr(recv_topk_weights), K,
+                                    _ptr(recv_src_metadata), cap, _stream(recv_x.device))
+    _check(st, "ep_write_padding_rows")

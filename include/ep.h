@@ -94,6 +94,10 @@ typedef struct {
      * and right after the pack kernel(s), for timing; NULL = none */
     void* event_pack_begin;
     void* event_pack_end;
+    /* added to the token index written to recv_src_metadata (0 normally); a
+     * GPU that holds tokens [o, o + T) of a larger batch passes o so that the
+     * metadata names tokens of the whole batch */
+    int32_t token_offset;
 } ep_dispatch_opts_t;
 
 /* The routing handle ep_dispatch fills and ep_combine reads (EPHandle of the
@@ -307,6 +311,28 @@ ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant,
 ep_status_t ep_group_limited_gating(const float* logits, int32_t T, int32_t E, int32_t n_group,
                                     int32_t topk_group, int32_t per_group, int64_t* topk_idx,
                                     float* topk_weights, int32_t* err, void* stream);
+
+/*
+ * Padding rows of a receive layout whose real rows were placed by another path
+ * (the multi-GPU exchange writes each source GPU's rows straight into a
+ * receiver's layout, and the receiver then fills the alignment padding that
+ * ep_dispatch would have written; comparative analysis section 3.1, expert
+ * alignment).  For each expert segment e < n_experts, the rows
+ * [psum[e-1] + counts[e], psum[e]) (psum[-1] = 0) get zero bytes in recv_x,
+ * zero bytes in recv_scales, recv_topk_idx -1, recv_topk_weights 0 and
+ * recv_src_metadata (-1, -1) -- the padding rows of ep_dispatch.
+ *   psum, counts        device int32 [n_experts]: inclusive prefix of the
+ *                       aligned counts, and the unaligned counts
+ *   recv_x              device, row_bytes per row (a multiple of 16, 16-byte aligned)
+ *   recv_scales         device, scale_row_bytes per row, or NULL
+ *   recv_topk_idx / recv_topk_weights  device [capacity, K], or NULL
+ *   recv_src_metadata   device int32 [capacity, 2], or NULL
+ * Rows at or past capacity are not written.  1 <= n_experts <= 1024.
+ */
+ep_status_t ep_write_padding_rows(const int32_t* psum, const int32_t* counts, int32_t n_experts, void* recv_x,
+                                  int64_t row_bytes, void* recv_scales, int64_t scale_row_bytes,
+                                  int32_t* recv_topk_idx, float* recv_topk_weights, int32_t K,
+                                  int32_t* recv_src_metadata, int64_t capacity, void* stream);
 
 /* Waits for `stream`, then copies the device status word to *host_status.
  * Returns EP_OK, or EP_ERR_CUDA if the wait or the copy failed. */
