@@ -52,7 +52,7 @@ def test_deepseek_v3_shapes(T, cuda_device):
     (64, 1, 1, 8, 517),        # one group: plain top-8
     (36, 6, 3, 2, 300),        # groups of 6 (scalar loads)
     (1024, 32, 2, 8, 257),     # K = 16, groups of 32
-    (256, 32, 32, 1, 64),      # every group kept, one expert each
+    (256, 16, 16, 1, 64),      # every group kept, one expert each (K = 16)
     (96, 32, 5, 3, 129),       # every expert of a kept group
     (12, 3, 2, 2, 1),
 ])
