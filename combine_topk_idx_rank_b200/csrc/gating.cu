@@ -44,10 +44,12 @@ __device__ __forceinline__ float sanitize(float x, int& bad) {
 
 template <int P>
 __device__ __forceinline__ void insert(float x, int e, float (&v)[P], int (&id)[P]) {
-    // carry (x, e) down the descending list; an empty slot (id < 0) takes it
+    // carry (x, e) down the list, kept in (larger value, lower id) order; an
+    // empty slot (id < 0) takes it.  A displaced entry carried further down
+    // may tie with a later entry by value, so the comparison includes the id.
 #pragma unroll
     for (int j = 0; j < P; ++j) {
-        if (id[j] < 0 || x > v[j]) {
+        if (id[j] < 0 || ahead(x, e, v[j], id[j])) {
             const float tv = v[j];
             const int te = id[j];
             v[j] = x;

@@ -1,12 +1,14 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
 benchmark times (capacity-bound buffers, no host sync inside dispatch).
 
-The oracle computes the layout and every slot for the whole routing (cheap),
-so those are compared in full.  Received rows and combined tokens are compared
-on a random sample of tokens the oracle computes one by one; in addition two
-properties are checked on every row: padding rows are all zero, and for bf16
-dispatch every received row equals its source token's row.
+Everything is compared in full, against the oracle's OpenMP build on every
+host core: the layout and every slot, every received row and scale of every
+token, and every combined token.  In addition two properties are checked on
+every row: padding rows are all zero, and for bf16 dispatch every received
+row equals its source token's row.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -18,6 +20,13 @@ from combine_topk_idx_rank_b200.workloads import CONFIGS, make_workload
 from gpu_parity import assert_combine_close, assert_layout_equal, to_dev, u8, u16
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def threaded_oracle():
+    oracle.use_threads(len(os.sched_getaffinity(0)))
+    yield
+    oracle.use_threads(1)
 
 
 @pytest.mark.parametrize("name", ["prefill", "decode", "qwen3", "longseq", "tiny"])
@@ -68,9 +77,8 @@ def test_full_size(name, cuda_device):
             assert torch.equal(bufs.recv_x.index_select(0, r).view(torch.int16),
                                x.index_select(0, t).view(torch.int16))
 
-    # sampled tokens: rows and scales against the oracle, one token at a time
-    rng = np.random.default_rng(1)
-    tok = np.sort(rng.choice(T, size=min(T, 96), replace=False)).astype(np.int32)
+    # every token's rows and scales against the oracle
+    tok = np.arange(T, dtype=np.int32)
     dst = s["dst_buffer_slot_idx"]
     sub = dst[tok]
     used = np.unique(sub[sub >= 0])
@@ -88,7 +96,7 @@ def test_full_size(name, cuda_device):
         gs = bufs.recv_scales.index_select(0, ridx).cpu().numpy()
         assert np.array_equal(gs.view(np.uint32), ref_s.view(np.uint32))
 
-    # combine on seeded expert outputs y; the oracle sees the sampled tokens' rows
+    # combine of every token on seeded expert outputs y
     g = torch.Generator(device=dev)
     g.manual_seed(99)
     y = torch.randn((bufs.recv_x.shape[0], H), generator=g, device=dev, dtype=torch.bfloat16)

@@ -2,10 +2,12 @@
 times besides the default one: the low-latency layout, cached dispatch, the
 combine of quantised expert outputs, MXFP4 dispatch and UE8M0 scale bytes.
 
-As in test_gpu_fullsize, the oracle computes the routing in full (cheap) and
-the rows, scales and combined tokens of a random sample of tokens, one token
-at a time; those are compared bit for bit.
+As in test_gpu_fullsize, everything is compared in full and bit for bit
+against the oracle's OpenMP build on every host core: the routing, and the
+rows, scales and combined tokens of every token.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -19,9 +21,16 @@ from gpu_parity import assert_combine_close, to_dev, u8, u16
 pytestmark = pytest.mark.gpu
 
 
-def _sample(T, n=96, seed=1):
-    rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(T, size=min(T, n), replace=False)).astype(np.int32)
+@pytest.fixture(autouse=True)
+def threaded_oracle():
+    oracle.use_threads(len(os.sched_getaffinity(0)))
+    yield
+    oracle.use_threads(1)
+
+
+def _sample(T):
+    """Every token (the rows below are compacted to those the tokens use)."""
+    return np.arange(T, dtype=np.int32)
 
 
 def _compact(dst, tok):
@@ -76,7 +85,7 @@ def test_full_size_low_latency_decode(cuda_device):
 @pytest.mark.parametrize("name", ["decode", "prefill"])
 def test_full_size_cached_dispatch(name, cuda_device):
     """A second dispatch with new activations and the first call's handle:
-    the sampled tokens' rows are the oracle's rows of the new x at the first
+    every token's rows are the oracle's rows of the new x at the first
     routing's slots; every padding row is zero again."""
     dev = cuda_device
     cfg = CONFIGS[name]
