@@ -92,7 +92,10 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             // x was written before this call's routing kernel started, so the
             // pack may read it while routing runs; a cached dispatch has no
             // routing kernel before it and waits for its predecessor first
-            pa.prefetch = after_routing ? 1 : 0;
+#ifndef EP_PACK_PREFETCH
+#define EP_PACK_PREFETCH 1   // 0: the staged pack waits for routing before it loads x
+#endif
+            pa.prefetch = (after_routing && EP_PACK_PREFETCH) ? 1 : 0;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }

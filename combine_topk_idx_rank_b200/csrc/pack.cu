@@ -873,7 +873,10 @@ cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
     return launch_dependent(k, dim3(grid), dim3(threads), 0, st, a);
 }
 
-constexpr size_t kStagedSmemMax = 200 * 1024;   // shared memory of one staged CTA, at most
+#ifndef EP_PACK_STAGED_SMEM_MAX
+#define EP_PACK_STAGED_SMEM_MAX (200 * 1024)   // shared memory of one staged CTA, at most (0: never staged)
+#endif
+constexpr size_t kStagedSmemMax = EP_PACK_STAGED_SMEM_MAX;
 
 // The staged kernel when every CTA's rows fit in shared memory in one wave
 // (decode-sized batches); returns cudaErrorNotSupported when they do not.
@@ -909,7 +912,7 @@ cudaError_t try_staged(const PackArgs& a, cudaStream_t st) {
 template <int QUANT, int G>
 cudaError_t staged_or_group(const PackArgs& a, int threads, cudaStream_t st) {
     constexpr int P = EP_PACK_GROUP_UPT;
-    if (a.staged) {
+    if (a.staged && kStagedSmemMax > 0) {
         const cudaError_t e = try_staged<QUANT, G>(a, st);
         if (e != cudaErrorNotSupported) return e;
     }
