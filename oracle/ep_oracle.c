@@ -269,6 +269,14 @@ int oracle_quantize_row(const uint16_t* x, int H, int quant, int quant_size, int
         scales[g] = s;
         for (int i = 0; i < quant_size; ++i) {
             float v = oracle_bf16_to_f32(x[g * quant_size + i]) / s;
+            /* A group whose maximum is infinite has an infinite scale, and an
+             * infinite x then gives inf / inf, a NaN whose sign IEEE 754 leaves
+             * open.  Reading: that NaN encodes as the positive FP8 NaN code
+             * S.1111.111 with S = 0, and as int8 0. */
+            if (isnan(v)) {
+                q[g * quant_size + i] = (quant == OR_QUANT_FP8) ? 0x7f : 0;
+                continue;
+            }
             if (quant == OR_QUANT_FP8) {
                 q[g * quant_size + i] = oracle_f32_to_e4m3(v);
             } else {

@@ -188,3 +188,21 @@ def test_rounds_equal_one_shot(quant, qs):
     o1 = oracle.combine(y, a["dst_buffer_slot_idx"], wl.topk_weights)
     o8 = oracle.combine(y, a["dst_buffer_slot_idx"], wl.topk_weights, cfg.num_ranks, 8)
     assert np.array_equal(o1, o8)
+
+
+def test_infinite_group_maximum():
+    """A group holding +-inf has an infinite scale: finite values quantise to
+    zero codes, and an infinite value gives inf / inf = NaN, whose sign IEEE
+    754 leaves open; the reading taken is the positive FP8 NaN code 0x7f, and
+    int8 0."""
+    row = np.zeros(128, np.uint16)
+    row[0] = 0x7F80           # +inf
+    row[1] = 0xFF80           # -inf
+    row[2] = 0x3F80           # 1.0
+    row[3] = 0xBF80           # -1.0
+    q, sc = oracle.quantize_row(row, "fp8", 128, False)
+    assert np.isinf(sc[0])
+    assert q[0] == 0x7F and q[1] == 0x7F
+    assert q[2] == 0x00 and q[3] == 0x80        # +0 and -0
+    q, _ = oracle.quantize_row(row, "int8", 128, False)
+    assert q[0] == 0 and q[1] == 0 and q[2] == 0 and q[3] == 0
