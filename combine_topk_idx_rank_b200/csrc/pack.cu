@@ -45,6 +45,9 @@
 #ifndef EP_PACK_STORE_HINT
 #define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
 #endif
+#ifndef EP_PACK_CODE_STORE
+#define EP_PACK_CODE_STORE 0   // quantised code stores: 0 default, 1 .cs, 2 L2 evict-first hint, 3 .wt
+#endif
 
 namespace ep {
 
@@ -85,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
-#if EP_PACK_LOAD_HINT || EP_PACK_STORE_HINT
+#if EP_PACK_LOAD_HINT || EP_PACK_STORE_HINT || EP_PACK_CODE_STORE == 2
 // L2 policy that marks lines for early eviction (rows are read or written once)
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t pol;
@@ -127,6 +130,23 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16 bytes of quantised codes to a received row.
+__device__ __forceinline__ void st_code_v4(void* p, uint4 v) {
+#if EP_PACK_CODE_STORE == 1
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+#elif EP_PACK_CODE_STORE == 2
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(l2_evict_first())
+                 : "memory");
+#elif EP_PACK_CODE_STORE == 3
+    asm volatile("st.global.wt.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+#else
+    st_v4(p, v);
+#endif
 }
 
 // Padding map from the handle: expert e's padding rows are
@@ -607,7 +627,7 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
                         if constexpr (QUANT == kQuantMxfp4) {
                             *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[j].x, q[j].y);
                         } else {
-                            st_v4(dst + 16 * (size_t)u, q[j]);
+                            st_code_v4(dst + 16 * (size_t)u, q[j]);
                         }
                         if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[j]);
                     }
