@@ -87,13 +87,11 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
-            pa.staged = 1;
-            pa.scales16 = aligned16(recv_scales);
             // x was written before this call's routing kernel started, so the
             // pack may read it while routing runs; a cached dispatch has no
             // routing kernel before it and waits for its predecessor first
 #ifndef EP_PACK_PREFETCH
-#define EP_PACK_PREFETCH 1   // 0: the staged pack waits for routing before it loads x
+#define EP_PACK_PREFETCH 1   // 0: the pipelined group pack waits for routing before it loads x
 #endif
             pa.prefetch = (after_routing && EP_PACK_PREFETCH) ? 1 : 0;
             s = cuda_status(launch_pack(pa, quant, st));

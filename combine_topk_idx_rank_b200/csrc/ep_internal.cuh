@@ -119,8 +119,6 @@ struct PackArgs {
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
     int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
-    int staged;                 // group quantisation may stage rows in shared memory
-    int scales16;               // recv_scales is 16-byte aligned (bulk stores of scale rows)
     int prefetch;               // x may be read before the routing kernel has finished (the pack
                                 // follows this call's routing, which started after x was written)
     int32_t* err;

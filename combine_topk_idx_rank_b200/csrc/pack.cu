@@ -653,132 +653,139 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
 }
 
 
-// ------------------------------------- group quantisation, staged (small T)
-// For batches whose quantised rows fit in shared memory (decode-sized
-// dispatch), every CTA owns J token rows (items b, b + grid, ...).  Before
-// waiting for routing it loads them, quantises them and keeps the codes and
-// scales in shared memory: none of that depends on routing, so it overlaps the
-// routing kernel (the pack is launched as its programmatic dependent; x was
-// written before routing started).  After the wait, threads 0..J*K-1 each issue
-// the bulk (TMA) stores of one staged row to one destination row.  The
-// launcher picks J >= the rows of every CTA, or the streaming group kernel
-// when they do not fit.
+// ------------------------------- group quantisation, TMA-pipelined rows
+// One token row per item (the whole row fits one pass: UPT x blockDim units).
+// The bf16 rows reach shared memory through bulk copies (cp.async.bulk with
+// an mbarrier per stage) issued S items ahead by thread 0, so each thread's
+// work per item is: read its units from the stage, quantise, store codes and
+// scales to the token's destination rows.  The first S rows are requested
+// before the wait for routing (x was written before routing started), and the
+// destination rows of item j + S are loaded into a register during item j and
+// published in shared memory during item j + 1.  Every wait is bounded.
 template <int QUANT, int G, int UPT>
-__global__ void __launch_bounds__(512, 2) k_pack_staged(PackArgs a, int J, int item_bytes) {
+__global__ void __launch_bounds__(512, 2) k_pack_group_tma(PackArgs a, int S, int stage_bytes) {
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
+    __shared__ int s_ok;
     constexpr int kLanes = G / 16;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     constexpr int kUnitBytes = QUANT == kQuantMxfp4 ? 8 : 16;   // code bytes of 16 channels
-    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
-    int* s_slot = reinterpret_cast<int*>(smem + (size_t)J * item_bytes);   // [J*K]
-    const int tid = threadIdx.x, bd = blockDim.x;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+    int* sslot = reinterpret_cast<int*>(mbar + S);                     // [S][kMaxTopk]
+    const int tid = threadIdx.x, bd = blockDim.x, K = a.K;
     const int U = a.H / 16;
-    const int K = a.K;
+    const uint32_t xrow = (uint32_t)a.H * 2;
     const int64_t row_bytes = (int64_t)U * kUnitBytes;
     const int nscales = a.H / G;
-    const int srb = nscales * (a.scale_bytes ? 1 : 4);                      // scale bytes per row
-    const bool scales_bulk = (srb & 15) == 0 && a.scales16;
     const int grid = gridDim.x;
     const int mine = a.n_tok_items > (int)blockIdx.x ? (a.n_tok_items - 1 - (int)blockIdx.x) / grid + 1 : 0;
+    const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.x);
 
-    auto token = [&](int j) {   // token of this CTA's j-th item
+    auto token = [&](int j) {
         return token_of_item((int)blockIdx.x + j * grid, a.tokens_per_rank, a.per_round, a.round);
     };
-    auto fetch = [&](int j, uint4 (&r)[UPT][2]) {
-        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)token(j) * a.H);
-#pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-            const int u = tid + i * bd;
-            if (u < U) {
-                r[i][0] = ld_nc_v4(xr + 2 * u);
-                r[i][1] = ld_nc_v4(xr + 2 * u + 1);
-            } else {
-                r[i][0] = r[i][1] = make_uint4(0, 0, 0, 0);
-            }
-        }
+    auto issue = [&](int j) {   // thread 0: bulk copy of item j's row into its stage
+        uint64_t* bar = &mbar[j % S];
+        mbar_expect_tx(bar, xrow);
+        bulk_load(smem + (size_t)(j % S) * stage_bytes, xb + (int64_t)token(j) * xrow, xrow, bar);
     };
-    // quantises one row held in registers into stage `st`
-    auto quantise = [&](int st, const uint4 (&r)[UPT][2]) {
-        uint8_t* codes = smem + (size_t)st * item_bytes;
-        uint8_t* scl = codes + row_bytes;
+    // thread 0 waits for stage j and tells the CTA (false: the bounded wait gave up)
+    auto landed = [&](int j) {
+        if (tid == 0) s_ok = mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1)) ? 1 : 0;
+        __syncthreads();
+        return s_ok != 0;
+    };
+    auto drain = [&](int issued_from, int issued_to) {   // thread 0: let issued copies land
+        if (tid == 0)
+            for (int j = issued_from; j < issued_to; ++j) mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1));
+        __syncthreads();
+    };
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(&mbar[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int pro = min(S, mine);
+    if (a.prefetch && tid == 0)
+        for (int j = 0; j < pro; ++j) issue(j);   // before routing has finished
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (routing_gave_up(a)) {
+        if (a.prefetch) drain(0, pro);
+        return;
+    }
+    if (!a.prefetch && tid == 0)
+        for (int j = 0; j < pro; ++j) issue(j);
+    for (int i = tid; i < pro * K; i += bd) {
+        const int j = i / K, k = i - j * K;
+        sslot[j * kMaxTopk + k] = checked_row(a, a.dst_slot[(int64_t)token(j) * K + k]);
+    }
+    int pending = -1;                             // destination row of item S (thread k < K)
+    if (tid < K && S < mine) pending = a.dst_slot[(int64_t)token(S) * K + tid];
+
+    for (int j = 0; j < mine; ++j) {
+        const int s = j % S;
+        if (!landed(j)) {
+            set_error(a.err, EP_ERR_TIMEOUT);
+            drain(j, min(mine, j + S));   // the copies issued so far land before the CTA exits
+            return;
+        }
+        mbar_try_wait(&mbar[s], (uint32_t)((j / S) & 1));   // completes at once: orders this thread's reads
+        const uint4* xs = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
+        uint4 q[UPT];
+        float sc[UPT];
 #pragma unroll
         for (int i = 0; i < UPT; ++i) {
             const int u = tid + i * bd;
             float f[16];
-            unpack16(r[i][0], r[i][1], f);
+            if (u < U) {
+                unpack16(xs[2 * u], xs[2 * u + 1], f);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) f[c] = 0.0f;
+            }
             float m = amax16(f);
 #pragma unroll
             for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (u < U) {
-                float sc;
-                if constexpr (QUANT == kQuantMxfp4) {
-                    sc = mx_scale(m);
-                    *reinterpret_cast<uint2*>(codes + 8 * (size_t)u) = quant16_fp4(f, sc);
-                } else {
-                    sc = finish_scale(m, kQmax, a.round_scale);
-                    *reinterpret_cast<uint4*>(codes + 16 * (size_t)u) = quant16<QUANT>(f, sc);
-                }
-                if ((u % kLanes) == 0) {
-                    if (a.scale_bytes) scl[u / kLanes] = ue8m0_of(sc);
-                    else reinterpret_cast<float*>(scl)[u / kLanes] = sc;
-                }
+            if constexpr (QUANT == kQuantMxfp4) {
+                sc[i] = mx_scale(m);
+                const uint2 c = quant16_fp4(f, sc[i]);
+                q[i] = make_uint4(c.x, c.y, 0, 0);
+            } else {
+                sc[i] = finish_scale(m, kQmax, a.round_scale);
+                q[i] = quant16<QUANT>(f, sc[i]);
             }
         }
-    };
-    // loads and quantises items [j0, j1) into stages 0.. (the next row's loads
-    // are issued before the current row is quantised)
-    auto stage_wave = [&](int j0, int j1) {
-        uint4 raw[UPT][2];
-        if (j0 < j1) fetch(j0, raw);
-        for (int j = j0; j < j1; ++j) {
-            uint4 nraw[UPT][2];
-            if (j + 1 < j1) fetch(j + 1, nraw);
-            quantise(j - j0, raw);
-            if (j + 1 < j1) {
+        for (int k = 0; k < K; ++k) {
+            const int slot = sslot[s * kMaxTopk + k];
+            if (slot < 0) continue;
+            uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
 #pragma unroll
-                for (int i = 0; i < UPT; ++i) {
-                    raw[i][0] = nraw[i][0];
-                    raw[i][1] = nraw[i][1];
+            for (int i = 0; i < UPT; ++i) {
+                const int u = tid + i * bd;
+                if (u < U) {
+                    if constexpr (QUANT == kQuantMxfp4) {
+                        *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[i].x, q[i].y);
+                    } else {
+                        st_code_v4(dst + 16 * (size_t)u, q[i]);
+                    }
+                    if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[i]);
                 }
             }
         }
-        fence_proxy_async_smem();   // the bulk stores read these bytes through the async proxy
-        __syncthreads();
-    };
-
-    // the launcher sizes J so that J >= this CTA's rows: one wave
-    const int n = min(J, mine);
-    if (a.prefetch) stage_wave(0, n);   // before routing has finished
-    grid_dependency_wait();
-    grid_launch_dependents();
-    if (routing_gave_up(a)) return;
-    if (!a.prefetch) stage_wave(0, n);
-
-    for (int i = tid; i < n * K; i += bd) {
-        const int j = i / K, k = i - j * K;
-        s_slot[i] = checked_row(a, a.dst_slot[(int64_t)token(j) * K + k]);
-    }
-    __syncthreads();
-    for (int i = tid; i < n * K; i += bd) {
-        const int slot = s_slot[i];
-        if (slot < 0) continue;
-        const uint8_t* src = smem + (size_t)(i / K) * item_bytes;
-        bulk_store(a.recv_x + (int64_t)slot * row_bytes, src, (uint32_t)row_bytes);
-        if (scales_bulk)
-            bulk_store(reinterpret_cast<uint8_t*>(a.recv_scales) + (int64_t)slot * srb, src + row_bytes,
-                       (uint32_t)srb);
-        bulk_commit();
-    }
-    if (!scales_bulk) {   // scale rows that are not a multiple of 16 bytes: plain stores
-        for (int i = tid; i < n * K * srb; i += bd) {
-            const int e = i / srb, b = i - e * srb;
-            const int slot = s_slot[e];
-            if (slot >= 0)
-                reinterpret_cast<uint8_t*>(a.recv_scales)[(int64_t)slot * srb + b] =
-                    smem[(size_t)(e / K) * item_bytes + row_bytes + b];
+        __syncthreads();   // stage s and its destination rows are free
+        if (j + S < mine) {
+            if (tid == 0) {
+                fence_proxy_async_smem();   // this CTA's reads of the stage come before the copy's writes
+                issue(j + S);
+            }
+            if (tid < K) {
+                sslot[s * kMaxTopk + tid] = checked_row(a, pending);
+                pending = j + S + 1 < mine ? a.dst_slot[(int64_t)token(j + S + 1) * K + tid] : -1;
+            }
         }
     }
-    bulk_wait_all();
 
     if (a.do_pad) {
         const int n_pad = build_pad_map(a, s_pad_base, s_pad_start, s_warp);
@@ -893,49 +900,29 @@ cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
     return launch_dependent(k, dim3(grid), dim3(threads), 0, st, a);
 }
 
-#ifndef EP_PACK_STAGED_SMEM_MAX
-#define EP_PACK_STAGED_SMEM_MAX (200 * 1024)   // shared memory of one staged CTA, at most (0: never staged)
+#ifndef EP_PACK_TMA_STAGES
+#define EP_PACK_TMA_STAGES 4   // bf16 rows in flight per CTA of the pipelined group pack (0: not used)
 #endif
-constexpr size_t kStagedSmemMax = EP_PACK_STAGED_SMEM_MAX;
 
-// The staged kernel when every CTA's rows fit in shared memory in one wave
-// (decode-sized batches); returns cudaErrorNotSupported when they do not.
+// The pipelined group kernel for rows of up to 1024 units (16384 channels).
 template <int QUANT, int G>
-cudaError_t try_staged(const PackArgs& a, cudaStream_t st) {
+cudaError_t launch_group_tma(const PackArgs& a, cudaStream_t st) {
     const int U = a.H / 16;
-    if (U > 1024) return cudaErrorNotSupported;
-    const int unit_bytes = QUANT == kQuantMxfp4 ? 8 : 16;
+    const int S = EP_PACK_TMA_STAGES;
     const int threads = min(512, round_up32(U <= 512 ? U : (U + 1) / 2));
-    const int nscales = a.H / G;
-    const int srb = nscales * (a.scale_bytes ? 1 : 4);
-    const int item_bytes = (int)(((size_t)U * unit_bytes + ((srb + 15) & ~15) + 15) & ~(size_t)15);
-    const int sms = device_sm_count();
-    auto kern = U <= 512 ? k_pack_staged<QUANT, G, 1> : k_pack_staged<QUANT, G, 2>;
-    // the most CTAs per SM whose rows (one wave) fit: J rows per CTA
-    for (int per_sm = 2048 / threads; per_sm >= 1; --per_sm) {
-        const int grid = sms * per_sm;
-        const int J = max(1, (a.n_tok_items + grid - 1) / grid);
-        const size_t smem = (size_t)J * item_bytes + (size_t)J * a.K * sizeof(int);
-        if (smem > kStagedSmemMax) continue;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        int fit = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem);
-        if (e != cudaSuccess) return e;
-        if (fit < per_sm) continue;
-        const int g = min(grid, max(1, a.n_tok_items));
-        return launch_dependent(kern, dim3(g), dim3(threads), smem, st, a, J, item_bytes);
-    }
-    return cudaErrorNotSupported;
+    const int stage_bytes = (a.H * 2 + 127) & ~127;
+    const size_t smem = (size_t)S * stage_bytes + S * sizeof(uint64_t) + (size_t)S * kMaxTopk * sizeof(int);
+    auto kern = U <= 512 ? k_pack_group_tma<QUANT, G, 1> : k_pack_group_tma<QUANT, G, 2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = min(max(1, a.n_tok_items), device_sm_count() * blocks_per_sm(kern, threads, smem));
+    return launch_dependent(kern, dim3(grid), dim3(threads), smem, st, a, S, stage_bytes);
 }
 
 template <int QUANT, int G>
-cudaError_t staged_or_group(const PackArgs& a, int threads, cudaStream_t st) {
+cudaError_t tma_or_group(const PackArgs& a, int threads, cudaStream_t st) {
     constexpr int P = EP_PACK_GROUP_UPT;
-    if (a.staged && kStagedSmemMax > 0) {
-        const cudaError_t e = try_staged<QUANT, G>(a, st);
-        if (e != cudaErrorNotSupported) return e;
-    }
+    if (EP_PACK_TMA_STAGES >= 2 && a.H / 16 <= 1024) return launch_group_tma<QUANT, G>(a, st);
     return run(k_pack_group<QUANT, G, P>, threads, a, st);
 }
 
@@ -946,15 +933,15 @@ cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
     const int threads = min(512 / P, round_up32((U + P - 1) / P));   // P units per thread
     if constexpr (QUANT == kQuantMxfp4) {
         if (a.quant_size != 32) return cudaErrorInvalidValue;
-        return staged_or_group<kQuantMxfp4, 32>(a, threads, st);
+        return tma_or_group<kQuantMxfp4, 32>(a, threads, st);
     }
     switch (a.quant_size) {
-        case 16: return staged_or_group<QUANT, 16>(a, threads, st);
-        case 32: return staged_or_group<QUANT, 32>(a, threads, st);
-        case 64: return staged_or_group<QUANT, 64>(a, threads, st);
-        case 128: return staged_or_group<QUANT, 128>(a, threads, st);
-        case 256: return staged_or_group<QUANT, 256>(a, threads, st);
-        case 512: return staged_or_group<QUANT, 512>(a, threads, st);
+        case 16: return tma_or_group<QUANT, 16>(a, threads, st);
+        case 32: return tma_or_group<QUANT, 32>(a, threads, st);
+        case 64: return tma_or_group<QUANT, 64>(a, threads, st);
+        case 128: return tma_or_group<QUANT, 128>(a, threads, st);
+        case 256: return tma_or_group<QUANT, 256>(a, threads, st);
+        case 512: return tma_or_group<QUANT, 512>(a, threads, st);
         default: return cudaErrorInvalidValue;
     }
 }
