@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libep.so")
 OBJDIR = os.path.join(HERE, "_build")
 SOURCES = ["routing.cu", "pack.cu", "combine.cu", "gating.cu", "padding.cu", "ep_api.cu", "ep_noalloc.cu"]
-HEADERS = ["ep_internal.cuh", os.path.join("..", "..", "include", "ep.h"),
+HEADERS = ["ep_internal.cuh", "quant.cuh", "tma.cuh", os.path.join("..", "..", "include", "ep.h"),
            os.path.join("..", "..", "include", "ep_testing.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")

@@ -26,15 +26,11 @@
 #include <cuda_fp8.h>
 
 #include "ep_internal.cuh"
+#include "quant.cuh"
+#include "tma.cuh"
 
 #ifndef EP_PACK_STAGES
 #define EP_PACK_STAGES 4
-#endif
-#ifndef EP_PACK_LOAD_HINT
-#define EP_PACK_LOAD_HINT 0    // 1: bulk loads of x rows carry an L2 evict-first policy
-#endif
-#ifndef EP_PACK_IEEE_DIV
-#define EP_PACK_IEEE_DIV 0     // 1: every quotient x / scale by the IEEE division
 #endif
 #ifndef EP_PACK_GROUP_UPT
 #define EP_PACK_GROUP_UPT 1          // 16-channel units per thread per pass of the group kernel
@@ -42,95 +38,12 @@
 #ifndef EP_PACK_GROUP_MIN_BLOCKS
 #define EP_PACK_GROUP_MIN_BLOCKS 2   // resident CTAs per SM the group kernel's registers must allow
 #endif
-#ifndef EP_PACK_STORE_HINT
-#define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
-#endif
-#ifndef EP_PACK_CODE_STORE
-#define EP_PACK_CODE_STORE 0   // quantised code stores: 0 default, 1 .cs, 2 L2 evict-first hint, 3 .wt
-#endif
 
 namespace ep {
 
 namespace {
 
-constexpr int kQuantFp8 = 1, kQuantInt8 = 2, kQuantMxfp4 = 3;
 constexpr int kBulkChunk = 16384;          // max bytes per pipeline stage
-constexpr unsigned kSpinLimit = 1u << 24;  // bounded mbarrier waits
-
-// ------------------------------------------------------ TMA bulk primitives
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Waits for phase `parity` of `bar`; false if the bounded wait gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (unsigned n = 0; n < kSpinLimit; ++n)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
-#if EP_PACK_LOAD_HINT || EP_PACK_STORE_HINT || EP_PACK_CODE_STORE == 2
-// L2 policy that marks lines for early eviction (rows are read or written once)
-__device__ __forceinline__ uint64_t l2_evict_first() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-#endif
-__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-#if EP_PACK_LOAD_HINT
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_u32(sdst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(l2_evict_first())
-        : "memory");
-#else
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(sdst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-#endif
-}
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-#if EP_PACK_STORE_HINT
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gdst),
-                 "r"(smem_u32(ssrc)), "r"(bytes), "l"(l2_evict_first())
-                 : "memory");
-#else
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-                 "r"(bytes)
-                 : "memory");
-#endif
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // 16 bytes of quantised codes to a received row.
 __device__ __forceinline__ void st_code_v4(void* p, uint4 v) {
@@ -201,114 +114,6 @@ __device__ __forceinline__ int64_t pad_row(int E, const int* s_base, const int* 
     return (int64_t)s_start[lo] + (p - s_base[lo]);
 }
 
-__device__ __forceinline__ float pow2_ceil_bits(float s) {
-    // s > 0 and normal: keep the exponent if the mantissa is zero, else bump it
-    const uint32_t u = __float_as_uint(s);
-    const uint32_t bumped = (u & 0xff800000u) + ((u & 0x007fffffu) ? 0x00800000u : 0u);
-    return __uint_as_float(bumped);
-}
-
-// Quotients x / s rounded to nearest even.  With r = RN(1/s), y = RN(x r) is
-// within one ulp of x / s, the remainder x - s y is exact in one fused
-// multiply-add, and the corrected y + r (x - s y) rounds to RN(x / s)
-// (Markstein's theorem on division with a fused multiply-add, IBM J. Res.
-// Develop. 34(1), 1990) -- provided nothing underflows: x and x / s must stay
-// well above the smallest normal.  So the corrected product is used when all
-// 16 inputs satisfy |x| >= max(2^-100, 2^-100 s); otherwise (a zero, a tiny
-// value, a NaN, or an infinite s) all 16 take the IEEE division.  Over every
-// pair of a bf16 x and a bf16 group maximum (scale = max(amax, 1e-4) / 448 or
-// / 127), the rule gives the same bits as the IEEE division.
-template <bool FAST>
-__device__ __forceinline__ void divide16(const float (&f)[16], float s, float (&v)[16]) {
-    if constexpr (!FAST || EP_PACK_IEEE_DIV) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(f[i], s);
-        return;
-    }
-    const float floor_ = fmaxf(0x1p-100f, __fmul_rn(0x1p-100f, s));
-    const float r = __frcp_rn(s);
-    bool fast = true;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        fast &= fabsf(f[i]) >= floor_;
-        const float y = __fmul_rn(f[i], r);
-        v[i] = __fmaf_rn(__fmaf_rn(-y, s, f[i]), r, y);
-    }
-    if (!fast) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(f[i], s);
-    }
-}
-
-// 16 channels -> 16 FP8 e4m3 (RNE, saturating) or int8 (RNE, clamped to
-// +-127) codes of x / s.  FAST: quotients by the rule of divide16 (the
-// per-token kernel, capped at 64 registers, keeps the plain IEEE division).
-template <int QUANT, bool FAST = true>
-__device__ __forceinline__ uint4 quant16(const float (&f)[16], float s) {
-    float v[16];
-    divide16<FAST>(f, s, v);
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if constexpr (QUANT == kQuantFp8) {
-            const __nv_fp8x2_storage_t lo =
-                __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i], v[4 * i + 1]), __NV_SATFINITE, __NV_E4M3);
-            const __nv_fp8x2_storage_t hi =
-                __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2], v[4 * i + 3]), __NV_SATFINITE, __NV_E4M3);
-            w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
-        } else {
-            uint32_t b = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                b |= (uint32_t)(max(-127, min(127, __float2int_rn(v[4 * i + j]))) & 0xff) << (8 * j);
-            w[i] = b;
-        }
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__device__ __forceinline__ void unpack16(uint4 lo, uint4 hi, float (&f)[16]) {
-    f[0] = bf16lo(lo.x); f[1] = bf16hi(lo.x); f[2] = bf16lo(lo.y); f[3] = bf16hi(lo.y);
-    f[4] = bf16lo(lo.z); f[5] = bf16hi(lo.z); f[6] = bf16lo(lo.w); f[7] = bf16hi(lo.w);
-    f[8] = bf16lo(hi.x); f[9] = bf16hi(hi.x); f[10] = bf16lo(hi.y); f[11] = bf16hi(hi.y);
-    f[12] = bf16lo(hi.z); f[13] = bf16hi(hi.z); f[14] = bf16lo(hi.w); f[15] = bf16hi(hi.w);
-}
-
-__device__ __forceinline__ float amax16(const float (&f)[16]) {
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(f[i]));
-    return m;
-}
-
-// MXFP4 shared scale of a 32-channel group: 2^(floor(log2 amax) - 2), 2 being
-// the largest exponent of E2M1 (the OCP MX conversion); amax floored at 1e-4.
-__device__ __forceinline__ float mx_scale(float amax) {
-    const uint32_t biased = (__float_as_uint(fmaxf(amax, 1e-4f)) >> 23) & 0xffu;
-    return __uint_as_float((biased - 2u) << 23);
-}
-
-// UE8M0 byte of a positive power of two: its biased exponent.
-__device__ __forceinline__ uint8_t ue8m0_of(float s) { return (uint8_t)((__float_as_uint(s) >> 23) & 0xffu); }
-
-// 16 channels -> 16 E2M1 codes, two per byte (even channel in the low nibble).
-__device__ __forceinline__ uint2 quant16_fp4(const float (&f)[16], float s) {
-    float v[16];
-    divide16<true>(f, s, v);
-    uint32_t w[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        w[h] = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const __nv_fp4x2_storage_t b = __nv_cvt_float2_to_fp4x2(
-                make_float2(v[8 * h + 2 * i], v[8 * h + 2 * i + 1]), __NV_E2M1, cudaRoundNearest);
-            w[h] |= (uint32_t)b << (8 * i);
-        }
-    }
-    return make_uint2(w[0], w[1]);
-}
-
 __device__ __forceinline__ void store_scale(const PackArgs& a, size_t idx, float s) {
     if (a.scale_bytes) reinterpret_cast<uint8_t*>(a.recv_scales)[idx] = ue8m0_of(s);
     else a.recv_scales[idx] = s;
@@ -319,11 +124,6 @@ __device__ __forceinline__ void zero_scales(const PackArgs& a, int64_t row, int 
         if (a.scale_bytes) reinterpret_cast<uint8_t*>(a.recv_scales)[row * nscales + j] = 0;
         else a.recv_scales[row * nscales + j] = 0.0f;
     }
-}
-
-__device__ __forceinline__ float finish_scale(float amax, float qmax, int round_scale) {
-    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), qmax);
-    return round_scale ? pow2_ceil_bits(s) : s;
 }
 
 // The routing kernel that this pack depends on stopped on its bounded wait:
