@@ -3,8 +3,6 @@
 // buffer belongs to the caller, nothing is allocated here.
 #include <stdio.h>
 
-#include <algorithm>
-
 #include "ep_internal.cuh"
 #include "../../include/ep_testing.h"
 
@@ -67,7 +65,7 @@ RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const
 // and unaligned counts.
 ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R, int quant, int quant_size,
                                const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
-                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st, bool after_routing) {
+                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st) {
     ep_status_t s;
     if (opts->event_pack_begin) {
         s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
@@ -89,13 +87,6 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
-            // x was written before this call's routing kernel started, so the
-            // pack may read it while routing runs; a cached dispatch has no
-            // routing kernel before it and waits for its predecessor first
-#ifndef EP_PACK_PREFETCH
-#define EP_PACK_PREFETCH 1   // 0: the pipelined group pack waits for routing before it loads x
-#endif
-            pa.prefetch = (after_routing && EP_PACK_PREFETCH) ? 1 : 0;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }
@@ -105,48 +96,6 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
         if (s) return s;
     }
     return EP_OK;
-}
-
-#ifndef EP_ROUTE_FUSE
-#define EP_ROUTE_FUSE 1   // 0: small batches are packed by the separate pack kernel
-#endif
-constexpr size_t kFuseSmemMax = 220 * 1024;   // dynamic shared memory of one fused routing CTA, at most
-
-// Small FP8 / int8 batches with groups of 128 channels (decode-sized) are
-// packed inside the routing kernel: the CTA that routes a chunk quantises the
-// chunk's rows while the grid barriers wait.  Sets r.fuse and its arguments
-// when the batch qualifies; the routing launcher still clears r.fuse when a
-// chunk per CTA does not fit on the device.
-void configure_fused_pack(RouteArgs& r, const void* x, int H, int quant, int quant_size, int A, int rounds,
-                          const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales, int64_t capacity) {
-    r.fuse = 0;
-    if (!EP_ROUTE_FUSE) return;
-    if (quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8) return;
-    if (quant_size != 128 || H % 128 != 0 || H > 8192 || rounds != 1 || A != 1) return;
-    if (r.T == 0 || capacity == 0 || recv_scales == nullptr) return;
-    const int scale_bytes = opts->scale_ue8m0 ? 1 : 0;
-    // enough bf16 rows in flight to cover a chunk's rows while the barriers wait
-    int stages = std::min(16, std::max(2, (64 * 1024) / (2 * H)));
-    const size_t base = (route_smem_bytes(r.E, r.K, r.R, r.log2_chunk) + 127) & ~(size_t)127;
-    while (stages > 2 && base + fuse_smem_bytes(r.log2_chunk, H, scale_bytes, stages) > kFuseSmemMax) --stages;
-    if (base + fuse_smem_bytes(r.log2_chunk, H, scale_bytes, stages) > kFuseSmemMax) return;
-    r.fuse = quant;   // EP_QUANT_FP8_E4M3 / EP_QUANT_INT8 are the kernels' quantisation kinds
-    r.x = static_cast<const uint16_t*>(x);
-    r.H = H;
-    r.round_scale = opts->round_scale ? 1 : 0;
-    r.scale_bytes = scale_bytes;
-    r.scales16 = aligned16(recv_scales);
-    r.recv_x = static_cast<uint8_t*>(recv_x);
-    r.recv_scales = recv_scales;
-    r.fuse_stages = stages;
-}
-
-// The pack events of a dispatch whose pack ran inside the routing kernel.
-ep_status_t record_fused_pack_events(const ep_dispatch_opts_t* opts, cudaStream_t st) {
-    ep_status_t s = EP_OK;
-    if (opts->event_pack_begin) s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
-    if (!s && opts->event_pack_end) s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_end), st));
-    return s;
 }
 
 // Quantisation options shared by ep_dispatch and ep_dispatch_cached.
@@ -271,12 +220,10 @@ ep_status_t dispatch_impl(const void* x, int32_t T, int32_t H, const int64_t* to
     r.err_out = h->err;
     r.stall = stall;
     r.token_offset = opts->token_offset;
-    configure_fused_pack(r, x, H, quant, quant_size, A, rounds, opts, recv_x, recv_scales, recv_capacity);
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-    if (r.fuse) return record_fused_pack_events(opts, st);
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, recv_capacity, h,
-                              st, true);
+                              st);
 }
 
 }  // namespace
@@ -375,11 +322,9 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
     r.cumulative = opts->cumulative_local_expert_recv_stats;
     r.err_out = h->err;
     r.token_offset = opts->token_offset;
-    configure_fused_pack(r, x, H, quant, quant_size, 1, rounds, opts, recv_x, recv_scales, rows);
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-    if (r.fuse) return record_fused_pack_events(opts, st);
-    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st, true);
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st);
 }
 
 ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dispatch_opts_t* opts,
@@ -401,7 +346,7 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
     if (h->recv_capacity > 0 && recv_x == nullptr) return EP_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, h->recv_capacity, h,
-                              static_cast<cudaStream_t>(stream), false);
+                              static_cast<cudaStream_t>(stream));
 }
 
 ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,

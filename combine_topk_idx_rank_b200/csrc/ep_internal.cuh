@@ -104,16 +104,6 @@ struct RouteArgs {
     // > 0 only from the test entry points: raises the first grid barrier's
     // target past the number of CTAs, so that no CTA can pass it
     unsigned stall;
-    // fused pack of small batches: 1 FP8 / 2 int8 (groups of 128), 0 none.  The
-    // launcher clears it when a chunk per CTA does not fit; the caller then
-    // launches the pack kernel itself.
-    int fuse;
-    const uint16_t* x;          // [T, H] bf16
-    int H, round_scale, scale_bytes, scales16;
-    uint8_t* recv_x;
-    float* recv_scales;
-    int fuse_stages;            // bf16 rows in flight per CTA
-    size_t fuse_smem_off;       // offset of the fused regions in dynamic shared memory (set by the launcher)
 };
 
 struct PackArgs {
@@ -129,8 +119,6 @@ struct PackArgs {
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
     int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
-    int prefetch;               // x may be read before the routing kernel has finished (the pack
-                                // follows this call's routing, which started after x was written)
     int32_t* err;
 };
 
@@ -174,9 +162,7 @@ struct PadArgs {
 };
 
 // Launchers (return the CUDA error of the launch).
-cudaError_t launch_route(RouteArgs& a, cudaStream_t st);   // may clear a.fuse
-size_t fuse_smem_bytes(int log2_chunk, int H, int scale_bytes, int stages);
-size_t route_smem_bytes(int E, int K, int R, int log2_chunk);
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t st);

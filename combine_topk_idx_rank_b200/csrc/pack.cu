@@ -453,153 +453,6 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
 }
 
 
-// ------------------------------- group quantisation, TMA-pipelined rows
-// One token row per item (the whole row fits one pass: UPT x blockDim units).
-// The bf16 rows reach shared memory through bulk copies (cp.async.bulk with
-// an mbarrier per stage) issued S items ahead by thread 0, so each thread's
-// work per item is: read its units from the stage, quantise, store codes and
-// scales to the token's destination rows.  The first S rows are requested
-// before the wait for routing (x was written before routing started), and the
-// destination rows of item j + S are loaded into a register during item j and
-// published in shared memory during item j + 1.  Every wait is bounded.
-template <int QUANT, int G, int UPT>
-__global__ void __launch_bounds__(512, 2) k_pack_group_tma(PackArgs a, int S, int stage_bytes) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
-    __shared__ int s_ok;
-    constexpr int kLanes = G / 16;
-    constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
-    constexpr int kUnitBytes = QUANT == kQuantMxfp4 ? 8 : 16;   // code bytes of 16 channels
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
-    int* sslot = reinterpret_cast<int*>(mbar + S);                     // [S][kMaxTopk]
-    const int tid = threadIdx.x, bd = blockDim.x, K = a.K;
-    const int U = a.H / 16;
-    const uint32_t xrow = (uint32_t)a.H * 2;
-    const int64_t row_bytes = (int64_t)U * kUnitBytes;
-    const int nscales = a.H / G;
-    const int grid = gridDim.x;
-    const int mine = a.n_tok_items > (int)blockIdx.x ? (a.n_tok_items - 1 - (int)blockIdx.x) / grid + 1 : 0;
-    const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.x);
-
-    auto token = [&](int j) {
-        return token_of_item((int)blockIdx.x + j * grid, a.tokens_per_rank, a.per_round, a.round);
-    };
-    auto issue = [&](int j) {   // thread 0: bulk copy of item j's row into its stage
-        uint64_t* bar = &mbar[j % S];
-        mbar_expect_tx(bar, xrow);
-        bulk_load(smem + (size_t)(j % S) * stage_bytes, xb + (int64_t)token(j) * xrow, xrow, bar);
-    };
-    // thread 0 waits for stage j and tells the CTA (false: the bounded wait gave up)
-    auto landed = [&](int j) {
-        if (tid == 0) s_ok = mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1)) ? 1 : 0;
-        __syncthreads();
-        return s_ok != 0;
-    };
-    auto drain = [&](int issued_from, int issued_to) {   // thread 0: let issued copies land
-        if (tid == 0)
-            for (int j = issued_from; j < issued_to; ++j) mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1));
-        __syncthreads();
-    };
-
-    if (tid == 0) {
-        for (int i = 0; i < S; ++i) mbar_init(&mbar[i], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    const int pro = min(S, mine);
-    if (a.prefetch && tid == 0)
-        for (int j = 0; j < pro; ++j) issue(j);   // before routing has finished
-    grid_dependency_wait();
-    grid_launch_dependents();
-    if (routing_gave_up(a)) {
-        if (a.prefetch) drain(0, pro);
-        return;
-    }
-    if (!a.prefetch && tid == 0)
-        for (int j = 0; j < pro; ++j) issue(j);
-    for (int i = tid; i < pro * K; i += bd) {
-        const int j = i / K, k = i - j * K;
-        sslot[j * kMaxTopk + k] = checked_row(a, a.dst_slot[(int64_t)token(j) * K + k]);
-    }
-    int pending = -1;                             // destination row of item S (thread k < K)
-    if (tid < K && S < mine) pending = a.dst_slot[(int64_t)token(S) * K + tid];
-
-    for (int j = 0; j < mine; ++j) {
-        const int s = j % S;
-        if (!landed(j)) {
-            set_error(a.err, EP_ERR_TIMEOUT);
-            drain(j, min(mine, j + S));   // the copies issued so far land before the CTA exits
-            return;
-        }
-        mbar_try_wait(&mbar[s], (uint32_t)((j / S) & 1));   // completes at once: orders this thread's reads
-        const uint4* xs = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
-        uint4 q[UPT];
-        float sc[UPT];
-#pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-            const int u = tid + i * bd;
-            float f[16];
-            if (u < U) {
-                unpack16(xs[2 * u], xs[2 * u + 1], f);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) f[c] = 0.0f;
-            }
-            float m = amax16(f);
-#pragma unroll
-            for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if constexpr (QUANT == kQuantMxfp4) {
-                sc[i] = mx_scale(m);
-                const uint2 c = quant16_fp4(f, sc[i]);
-                q[i] = make_uint4(c.x, c.y, 0, 0);
-            } else {
-                sc[i] = finish_scale(m, kQmax, a.round_scale);
-                q[i] = quant16<QUANT>(f, sc[i]);
-            }
-        }
-        for (int k = 0; k < K; ++k) {
-            const int slot = sslot[s * kMaxTopk + k];
-            if (slot < 0) continue;
-            uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
-#pragma unroll
-            for (int i = 0; i < UPT; ++i) {
-                const int u = tid + i * bd;
-                if (u < U) {
-                    if constexpr (QUANT == kQuantMxfp4) {
-                        *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[i].x, q[i].y);
-                    } else {
-                        st_code_v4(dst + 16 * (size_t)u, q[i]);
-                    }
-                    if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[i]);
-                }
-            }
-        }
-        __syncthreads();   // stage s and its destination rows are free
-        if (j + S < mine) {
-            if (tid == 0) {
-                fence_proxy_async_smem();   // this CTA's reads of the stage come before the copy's writes
-                issue(j + S);
-            }
-            if (tid < K) {
-                sslot[s * kMaxTopk + tid] = checked_row(a, pending);
-                pending = j + S + 1 < mine ? a.dst_slot[(int64_t)token(j + S + 1) * K + tid] : -1;
-            }
-        }
-    }
-
-    if (a.do_pad) {
-        const int n_pad = build_pad_map(a, s_pad_base, s_pad_start, s_warp);
-        for (int p = blockIdx.x; p < n_pad; p += grid) {
-            const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, p);
-            if (row >= 0 && row < a.capacity) {
-                uint4* dst = reinterpret_cast<uint4*>(a.recv_x + (size_t)row * row_bytes);
-                for (size_t v = tid; v < (size_t)row_bytes / 16; v += bd) st_v4(dst + v, make_uint4(0, 0, 0, 0));
-                zero_scales(a, row, nscales);
-            }
-        }
-    }
-}
-
 // ----------------------------------------------- per-token quantisation (G=H)
 // The whole row stays in registers (UPT units of 16 channels per thread) while
 // the block reduces its amax.
@@ -700,32 +553,6 @@ cudaError_t run(Kern k, int threads, const PackArgs& a, cudaStream_t st) {
     return launch_dependent(k, dim3(grid), dim3(threads), 0, st, a);
 }
 
-#ifndef EP_PACK_TMA_STAGES
-#define EP_PACK_TMA_STAGES 4   // bf16 rows in flight per CTA of the pipelined group pack (0: not used)
-#endif
-
-// The pipelined group kernel for rows of up to 1024 units (16384 channels).
-template <int QUANT, int G>
-cudaError_t launch_group_tma(const PackArgs& a, cudaStream_t st) {
-    const int U = a.H / 16;
-    const int S = EP_PACK_TMA_STAGES;
-    const int threads = min(512, round_up32(U <= 512 ? U : (U + 1) / 2));
-    const int stage_bytes = (a.H * 2 + 127) & ~127;
-    const size_t smem = (size_t)S * stage_bytes + S * sizeof(uint64_t) + (size_t)S * kMaxTopk * sizeof(int);
-    auto kern = U <= 512 ? k_pack_group_tma<QUANT, G, 1> : k_pack_group_tma<QUANT, G, 2>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int grid = min(max(1, a.n_tok_items), device_sm_count() * blocks_per_sm(kern, threads, smem));
-    return launch_dependent(kern, dim3(grid), dim3(threads), smem, st, a, S, stage_bytes);
-}
-
-template <int QUANT, int G>
-cudaError_t tma_or_group(const PackArgs& a, int threads, cudaStream_t st) {
-    constexpr int P = EP_PACK_GROUP_UPT;
-    if (EP_PACK_TMA_STAGES >= 2 && a.H / 16 <= 1024) return launch_group_tma<QUANT, G>(a, st);
-    return run(k_pack_group<QUANT, G, P>, threads, a, st);
-}
-
 template <int QUANT>
 cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
     constexpr int P = EP_PACK_GROUP_UPT;
@@ -733,15 +560,15 @@ cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
     const int threads = min(512 / P, round_up32((U + P - 1) / P));   // P units per thread
     if constexpr (QUANT == kQuantMxfp4) {
         if (a.quant_size != 32) return cudaErrorInvalidValue;
-        return tma_or_group<kQuantMxfp4, 32>(a, threads, st);
+        return run(k_pack_group<kQuantMxfp4, 32, P>, threads, a, st);
     }
     switch (a.quant_size) {
-        case 16: return tma_or_group<QUANT, 16>(a, threads, st);
-        case 32: return tma_or_group<QUANT, 32>(a, threads, st);
-        case 64: return tma_or_group<QUANT, 64>(a, threads, st);
-        case 128: return tma_or_group<QUANT, 128>(a, threads, st);
-        case 256: return tma_or_group<QUANT, 256>(a, threads, st);
-        case 512: return tma_or_group<QUANT, 512>(a, threads, st);
+        case 16: return run(k_pack_group<QUANT, 16, P>, threads, a, st);
+        case 32: return run(k_pack_group<QUANT, 32, P>, threads, a, st);
+        case 64: return run(k_pack_group<QUANT, 64, P>, threads, a, st);
+        case 128: return run(k_pack_group<QUANT, 128, P>, threads, a, st);
+        case 256: return run(k_pack_group<QUANT, 256, P>, threads, a, st);
+        case 512: return run(k_pack_group<QUANT, 512, P>, threads, a, st);
         default: return cudaErrorInvalidValue;
     }
 }

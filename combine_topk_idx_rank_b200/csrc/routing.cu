@@ -21,8 +21,6 @@
 //      outputs and the status word.
 // No sort, no global atomics except the barrier counter.
 #include "ep_internal.cuh"
-#include "quant.cuh"
-#include "tma.cuh"
 
 namespace ep {
 
@@ -36,20 +34,14 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 
-// The grid barrier in two halves, so that a CTA can do work that does not
-// depend on the other CTAs between its arrival and its wait: grid_arrive
-// publishes this CTA's writes and counts it in; grid_wait polls (bounded) until
-// `target` CTAs have arrived.
-__device__ __forceinline__ void grid_arrive(unsigned* counter) {
+// Grid-wide barrier over a counter that was zero at launch; `target` is
+// gridDim.x times the barrier's ordinal.  False if the wait gave up (after
+// kBarrierTimeoutNs of the global timer).
+__device__ bool grid_barrier(unsigned* counter, unsigned target, int* s_flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         atomicAdd(counter, 1u);
-    }
-}
-__device__ bool grid_wait(unsigned* counter, unsigned target, int* s_flag) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
         int ok = 1;
         const unsigned long long t0 = global_ns();
         for (;;) {
@@ -124,17 +116,10 @@ __device__ int block_exclusive_scan_E(const int* in, int* out, int E, int* s_war
 
 }  // namespace
 
-// FQ (fused pack of small batches, FP8 / int8 with groups of 128 channels):
-// each CTA routes exactly one chunk and also packs that chunk's tokens.  Their
-// bf16 rows stream into a ring of shared-memory stages by bulk copies issued
-// from the kernel's start; the CTA quantises them into shared memory between
-// its arrival at each grid barrier and its wait there, and once phase 3 has
-// assigned the chunk's rows it bulk-stores every token's codes and scales to
-// each of its rows.
-template <int KT, int FQ>
-__global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteArgs a) {
+template <int KT>
+__global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     grid_launch_dependents();   // the pack kernel may be scheduled; it waits for our results
-    extern __shared__ __align__(128) int32_t smem[];
+    extern __shared__ int32_t smem[];
     const int E = a.E, K = KT > 0 ? KT : a.K, R = a.R, L = a.L;
     const int C = 1 << a.log2_chunk;
     int32_t* wh = smem;                               // [8][E] per-warp running counts
@@ -160,96 +145,6 @@ __global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteA
     // with one chunk per CTA its ids, weights and ranks stay in shared memory
     // from phase 1 to phase 3; otherwise phase 3 reloads them
     const bool resident = a.nchunks <= G;
-
-    // ------------------------------------------------------ fused pack state
-    // (FQ only; the host picks it when every chunk has its own CTA)
-    constexpr int kFuseLanes = 128 / 16;                       // lanes of one 128-channel group
-    uint8_t* f_base = reinterpret_cast<uint8_t*>(smem) + a.fuse_smem_off;
-    const int f_U = a.H / 16;                                  // 16-channel units per row
-    const int64_t f_row = (int64_t)a.H;                        // code bytes per row
-    const int f_srb = (a.H / 128) * (a.scale_bytes ? 1 : 4);   // scale bytes per row
-    const int f_srb16 = (f_srb + 15) & ~15;
-    const int f_xrow = a.H * 2;                                // bf16 bytes per row
-    uint8_t* f_codes = f_base;                                 // [C][H]
-    uint8_t* f_scales = f_codes + (size_t)C * f_row;           // [C][f_srb16]
-    uint8_t* f_stage = f_scales + (size_t)C * f_srb16;         // [S][2H]
-    uint64_t* f_mbar = reinterpret_cast<uint64_t*>(f_stage + (size_t)a.fuse_stages * f_xrow);
-    const int f_S = a.fuse_stages;
-    const int f_chunk = blockIdx.x;                            // resident: chunk = CTA
-    const bool f_mine = FQ != 0 && f_chunk < a.nchunks;
-    const int f_t0 = f_mine ? (f_chunk / a.chunks_per_rank) * a.tokens_per_rank + (f_chunk % a.chunks_per_rank) * C : 0;
-    const int f_nt = f_mine ? min(C, a.tokens_per_rank - (f_chunk % a.chunks_per_rank) * C) : 0;
-    int f_issued = 0;                                          // tokens whose bulk copy is issued (thread 0)
-    int f_waited = 0;                                          // tokens whose copy thread 0 saw land
-    int* s_fok = s_misc + 34;                                  // 0 once a fused wait gave up
-    auto f_issue = [&](int tl) {                               // thread 0
-        uint64_t* bar = &f_mbar[tl % f_S];
-        mbar_expect_tx(bar, (uint32_t)f_xrow);
-        bulk_load(f_stage + (size_t)(tl % f_S) * f_xrow,
-                  reinterpret_cast<const uint8_t*>(a.x) + (int64_t)(f_t0 + tl) * f_xrow, (uint32_t)f_xrow, bar);
-    };
-    // quantises tokens [tl0, tl1) of the chunk from their stages into f_codes / f_scales
-    auto f_quantise = [&](int tl0, int tl1) {
-        for (int tl = tl0; tl < tl1; ++tl) {
-            const int st = tl % f_S;
-            const uint32_t par = (uint32_t)((tl / f_S) & 1);
-            if (tid == 0 && *s_fok) {
-                *s_fok = mbar_wait(&f_mbar[st], par) ? 1 : 0;
-                if (*s_fok) f_waited = tl + 1;
-            }
-            __syncthreads();
-            if (!*s_fok) return;
-            mbar_try_wait(&f_mbar[st], par);   // completes at once: orders this thread's reads
-            const uint4* xs = reinterpret_cast<const uint4*>(f_stage + (size_t)st * f_xrow);
-            uint8_t* codes = f_codes + (size_t)tl * f_row;
-            uint8_t* scl = f_scales + (size_t)tl * f_srb16;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {   // 16-channel units tid and tid + 256 (rows of up to 8192 channels)
-                const int u = tid + i * kRouteThreads;
-                float f[16];
-                if (u < f_U) {
-                    unpack16(xs[2 * u], xs[2 * u + 1], f);
-                } else {
-#pragma unroll
-                    for (int c2 = 0; c2 < 16; ++c2) f[c2] = 0.0f;
-                }
-                float m = amax16(f);
-#pragma unroll
-                for (int o = kFuseLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (u < f_U) {
-                    const float sc = finish_scale(m, FQ == kQuantFp8 ? 448.0f : 127.0f, a.round_scale);
-                    *reinterpret_cast<uint4*>(codes + 16 * (size_t)u) = quant16<FQ == kQuantFp8 ? kQuantFp8 : kQuantInt8>(f, sc);
-                    if ((u % kFuseLanes) == 0) {
-                        if (a.scale_bytes) scl[u / kFuseLanes] = ue8m0_of(sc);
-                        else reinterpret_cast<float*>(scl)[u / kFuseLanes] = sc;
-                    }
-                }
-            }
-            __syncthreads();   // stage st is free
-            if (tid == 0 && tl + f_S < f_nt) {
-                fence_proxy_async_smem();
-                f_issue(tl + f_S);
-                ++f_issued;
-            }
-        }
-    };
-    // thread 0: every copy issued but not yet seen to land (at most one per
-    // stage, each in its stage's latest phase) lands before the CTA exits
-    auto f_drain = [&]() {
-        if (FQ != 0 && tid == 0)
-            for (int tl = f_waited; tl < f_issued; ++tl) mbar_wait(&f_mbar[tl % f_S], (uint32_t)((tl / f_S) & 1));
-        __syncthreads();
-    };
-    if (FQ != 0) {
-        if (tid == 0) {
-            *s_fok = 1;
-            for (int i = 0; i < f_S; ++i) mbar_init(&f_mbar[i], 1);
-            fence_mbar_init();
-            for (int tl = 0; tl < min(f_S, f_nt); ++tl) f_issue(tl);   // x is ready: written before this call
-            f_issued = min(f_S, f_nt);
-        }
-        __syncthreads();
-    }
 
     // ---------------------------------------------------------------- phase 1
     // the status word of this call starts clear; every later error is first-wins
@@ -340,11 +235,8 @@ __global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteA
         if (tid == 0) a.chunk_err[c] = *s_err;
         __syncthreads();
     }
-    grid_arrive(a.barrier);
-    if (FQ != 0) f_quantise(0, f_nt / 2);   // while the other CTAs arrive
-    if (!grid_wait(a.barrier, (unsigned)G + a.stall, s_flag)) {
+    if (!grid_barrier(a.barrier, (unsigned)G + a.stall, s_flag)) {
         if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
-        f_drain();
         return;
     }
 
@@ -382,14 +274,8 @@ __global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteA
             if (lane == 0) a.col_total[col] = carry;
         }
     }
-    grid_arrive(a.barrier);
-    if (FQ != 0) {
-        f_quantise(f_nt / 2, f_nt);
-        fence_proxy_async_smem();   // the codes are read by bulk stores after phase 3
-    }
-    if (!grid_wait(a.barrier, 2u * G, s_flag)) {
+    if (!grid_barrier(a.barrier, 2u * G, s_flag)) {
         if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
-        f_drain();
         return;
     }
 
@@ -470,7 +356,6 @@ __global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteA
                 }
             }
             a.dst_slot[e0 + i] = slot;
-            if (FQ != 0) s_rank[i] = slot;   // the fused stores below read it
             if (slot < 0) continue;
             reinterpret_cast<int2*>(a.recv_meta)[slot] = make_int2(a.token_offset + t0 + tl, k);
             const int rdst = rank_of(e, L, shL);
@@ -505,37 +390,6 @@ __global__ void __launch_bounds__(kRouteThreads, FQ != 0 ? 1 : 3) k_route(RouteA
                 }
             }
         }
-    }
-    if (FQ != 0 && f_mine) {
-        // fused pack: every entry's codes and scales from shared memory to its row
-        __syncthreads();
-        if (*s_fok) {
-            const bool scales_bulk = (f_srb & 15) == 0 && a.scales16;
-            const int ne = f_nt * K;
-            for (int i = tid; i < ne; i += kRouteThreads) {
-                const int slot = s_rank[i];
-                if (slot < 0) continue;
-                const uint8_t* src = f_codes + (size_t)(i / K) * f_row;
-                bulk_store(a.recv_x + (int64_t)slot * f_row, src, (uint32_t)f_row);
-                if (scales_bulk)
-                    bulk_store(reinterpret_cast<uint8_t*>(a.recv_scales) + (int64_t)slot * f_srb,
-                               f_scales + (size_t)(i / K) * f_srb16, (uint32_t)f_srb);
-                bulk_commit();
-            }
-            if (!scales_bulk) {
-                for (int i = tid; i < ne * f_srb; i += kRouteThreads) {
-                    const int en = i / f_srb, b = i - en * f_srb;
-                    const int slot = s_rank[en];
-                    if (slot >= 0)
-                        reinterpret_cast<uint8_t*>(a.recv_scales)[(int64_t)slot * f_srb + b] =
-                            f_scales[(size_t)(en / K) * f_srb16 + b];
-                }
-            }
-            bulk_wait_all();
-        } else if (tid == 0) {
-            set_error(a.err_out, EP_ERR_TIMEOUT);   // a row never landed: nothing of this chunk is stored
-        }
-        f_drain();
     }
     if (a.ll_M) {
         // per (expert, source rank): (first row of the rank's block << 32) | entries
@@ -573,31 +427,18 @@ size_t route_smem_bytes(int E, int K, int R, int log2_chunk) {
            (size_t)C * R;
 }
 
-// Shared memory of the fused pack's regions: codes, scales, row stages and
-// their mbarriers.
-size_t fuse_smem_bytes(int log2_chunk, int H, int scale_bytes, int stages) {
-    const int C = 1 << log2_chunk;
-    const size_t srb16 = (size_t)(((H / 128) * (scale_bytes ? 1 : 4) + 15) & ~15);
-    return (size_t)C * H + (size_t)C * srb16 + (size_t)stages * H * 2 + (size_t)stages * sizeof(uint64_t);
-}
-
 namespace {
 
-template <int KT, int FQ>
-cudaError_t launch_route_k(RouteArgs& a, cudaStream_t st) {
-    size_t smem = route_smem_bytes(a.E, a.K, a.R, a.log2_chunk);
-    if (FQ != 0) {
-        a.fuse_smem_off = (smem + 127) & ~(size_t)127;
-        smem = a.fuse_smem_off + fuse_smem_bytes(a.log2_chunk, a.H, a.scale_bytes, a.fuse_stages);
-    }
-    cudaError_t e = cudaFuncSetAttribute(k_route<KT, FQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int KT>
+cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
+    const size_t smem = route_smem_bytes(a.E, a.K, a.R, a.log2_chunk);
+    cudaError_t e = cudaFuncSetAttribute(k_route<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_route<KT, FQ>, kRouteThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_route<KT>, kRouteThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int resident = per_sm * device_sm_count();
-    if (FQ != 0 && a.nchunks > resident) return cudaErrorNotSupported;   // a chunk per CTA is required
     const int grid = max(1, min(a.nchunks, resident));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -609,32 +450,20 @@ cudaError_t launch_route_k(RouteArgs& a, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_route<KT, FQ>, a);
-}
-
-template <int FQ>
-cudaError_t launch_route_q(RouteArgs& a, cudaStream_t st) {
-    switch (a.vector_ok ? a.K : 0) {
-        case 4: return launch_route_k<4, FQ>(a, st);
-        case 8: return launch_route_k<8, FQ>(a, st);
-        case 16: return launch_route_k<16, FQ>(a, st);
-        default: return launch_route_k<0, FQ>(a, st);
-    }
+    return cudaLaunchKernelEx(&cfg, k_route<KT>, a);
 }
 
 }  // namespace
 
-cudaError_t launch_route(RouteArgs& a, cudaStream_t st) {
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.barrier, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return e;
-    if (a.fuse == kQuantFp8 || a.fuse == kQuantInt8) {
-        e = a.fuse == kQuantFp8 ? launch_route_q<kQuantFp8>(a, st) : launch_route_q<kQuantInt8>(a, st);
-        if (e != cudaErrorNotSupported) return e;
-        cudaGetLastError();   // not launched; route without the fused pack
-        a.fuse = 0;
+    switch (a.vector_ok ? a.K : 0) {
+        case 4: return launch_route_k<4>(a, st);
+        case 8: return launch_route_k<8>(a, st);
+        case 16: return launch_route_k<16>(a, st);
+        default: return launch_route_k<0>(a, st);
     }
-    a.fuse = 0;
-    return launch_route_q<0>(a, st);
 }
 
 }  // namespace ep
