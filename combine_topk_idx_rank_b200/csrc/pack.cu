@@ -354,8 +354,16 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
     const int n_tok = a.n_tok_items * passes;
     const int n_items = n_tok + n_pad;
 
-    // item -> token, and the first unit of its pass
+    // item -> token, and the first unit of its pass; with one pass per row and
+    // one round (every workload but the longest rows and rounds) the item is
+    // the token, with no division
+    const bool direct = passes == 1 && a.per_round == a.tokens_per_rank;
     auto locate = [&](int item, int& t, int& u0) {
+        if (direct) {
+            t = item;
+            u0 = 0;
+            return;
+        }
         const int ti = item / passes;
         u0 = (item - ti * passes) * per_pass;
         t = token_of_item(ti, a.tokens_per_rank, a.per_round, a.round);

@@ -14,6 +14,9 @@
 #ifndef EP_PACK_IEEE_DIV
 #define EP_PACK_IEEE_DIV 0     // 1: every quotient x / scale by the IEEE division
 #endif
+#ifndef EP_QUANT_PAIRED
+#define EP_QUANT_PAIRED 1      // 1: the corrected quotients on packed fp32 pairs
+#endif
 
 namespace ep {
 namespace {
@@ -48,11 +51,29 @@ __device__ __forceinline__ void divide16(const float (&f)[16], float s, float (&
     const float r = __frcp_rn(s);
     bool fast = true;
 #pragma unroll
+    for (int i = 0; i < 16; ++i) fast &= fabsf(f[i]) >= floor_;
+#if EP_QUANT_PAIRED
+    // the same three correctly rounded operations on pairs of lanes (packed
+    // fp32 x2 arithmetic of sm_100): y = x r, e = y (-s) + x, v = e r + y
+    uint64_t r2, ns2;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r2) : "f"(r), "f"(r));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ns2) : "f"(-s), "f"(-s));
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        uint64_t x2, y2, e2, v2;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(x2) : "f"(f[i]), "f"(f[i + 1]));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y2) : "l"(x2), "l"(r2));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e2) : "l"(y2), "l"(ns2), "l"(x2));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v2) : "l"(e2), "l"(r2), "l"(y2));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(v[i]), "=f"(v[i + 1]) : "l"(v2));
+    }
+#else
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
-        fast &= fabsf(f[i]) >= floor_;
         const float y = __fmul_rn(f[i], r);
         v[i] = __fmaf_rn(__fmaf_rn(-y, s, f[i]), r, y);
     }
+#endif
     if (!fast) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(f[i], s);
