@@ -87,6 +87,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.quant_size = quant_size; pa.round_scale = opts->round_scale ? 1 : 0;
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
+            pa.x32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;   // rows of H % 16 == 0 channels stay aligned
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }
@@ -403,6 +404,7 @@ ep_status_t ep_group_limited_gating(const float* logits, int32_t T, int32_t E, i
     g.logits = logits;
     g.T = T; g.E = E; g.n_group = n_group; g.topk_group = topk_group; g.per_group = per_group;
     g.vec_ok = aligned16(logits) && E % 4 == 0;
+    g.vec8_ok = (reinterpret_cast<uintptr_t>(logits) & 31u) == 0 && E % 8 == 0;
     g.topk_idx = topk_idx; g.topk_weights = topk_weights;
     g.err = err;
     return cuda_status(launch_gate(g, static_cast<cudaStream_t>(stream)));

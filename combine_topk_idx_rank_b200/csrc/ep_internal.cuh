@@ -119,6 +119,7 @@ struct PackArgs {
     int tokens_per_rank, per_round, round, n_tok_items, do_pad;
     int quant_size, round_scale;
     int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
+    int x32;                    // x is 32-byte aligned: a 16-channel unit is one 32-byte load
     int32_t* err;
 };
 
@@ -141,6 +142,7 @@ struct GateArgs {
     int64_t T;
     int E, n_group, topk_group, per_group;
     int vec_ok;                 // logits 16-byte aligned (rows of E % 4 == 0 floats)
+    int vec8_ok;                // logits 32-byte aligned and E % 8 == 0
     int64_t* topk_idx;          // [T, K]
     float* topk_weights;        // [T, K]
     int32_t* err;               // [1] status word (cleared by the launch)
@@ -212,6 +214,14 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
     return r;
+}
+
+// 32-byte load (sm_100 256-bit global load) that does not allocate in L1; p
+// must be 32-byte aligned.  A warp of these reads 1 KB of whole sectors.
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint4& lo, uint4& hi) {
+    asm("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+        : "l"(p));
 }
 
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {

@@ -16,10 +16,11 @@
 //
 // One warp per token.  Lane g owns group g: it streams the group's S logits
 // (16-byte loads when S % 4 == 0) through a sorted per_group-entry insertion
-// list, then sums the list for the group's score.  The warp keeps the
-// topk_group best groups by repeated shuffle argmax; the chosen lanes write
-// their entries to shared memory, and lanes 0..K-1 each take one entry, count
-// the entries ahead of it (its output position), and compute its weight.
+// list, then sums the list for the group's score.  Each lane counts the groups
+// ahead of its own (one shuffle per group, all independent); the lanes of the
+// topk_group best groups write their entries to shared memory, and lanes
+// 0..K-1 each take one entry, count the entries ahead of it (its output
+// position), and compute its weight.
 // Non-finite logits set EP_ERR_NONFINITE; they are then ordered as -inf (NaN)
 // or +-inf so that the outputs stay K distinct in-range ids.
 #include <math.h>
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(kGateWarps * 32) k_gate(GateArgs a) {
     const int S = a.E / a.n_group;
     const int K = a.topk_group * P;
     const bool vec = (S & 3) == 0 && a.vec_ok;
+    const bool vec8 = (S & 7) == 0 && a.vec8_ok;
     for (int64_t t = (int64_t)blockIdx.x * kGateWarps + warp; t < a.T; t += (int64_t)gridDim.x * kGateWarps) {
         const float* row = a.logits + t * a.E;
         // 1. the group's per_group best experts and its score (lane g = group g)
@@ -83,7 +85,17 @@ __global__ void __launch_bounds__(kGateWarps * 32) k_gate(GateArgs a) {
         const bool owner = lane < a.n_group;
         if (owner) {
             const int e0 = lane * S;
-            if (vec) {
+            if (vec8) {   // 32-byte loads: a warp reads whole sectors
+                for (int i = 0; i < S / 8; ++i) {
+                    uint4 lo, hi;
+                    ld_nc_v8(row + e0 + 8 * i, lo, hi);
+                    const float q[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z),
+                                        __uint_as_float(lo.w), __uint_as_float(hi.x), __uint_as_float(hi.y),
+                                        __uint_as_float(hi.z), __uint_as_float(hi.w)};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) insert<P>(sanitize(q[c], bad), e0 + 8 * i + c, v, id);
+                }
+            } else if (vec) {
                 const float4* p = reinterpret_cast<const float4*>(row + e0);
 #pragma unroll 2
                 for (int i = 0; i < S / 4; ++i) {
@@ -102,28 +114,20 @@ __global__ void __launch_bounds__(kGateWarps * 32) k_gate(GateArgs a) {
 #pragma unroll
         for (int j = 1; j < P; ++j) score = score + v[j];
         if (score != score) score = -INFINITY;   // +inf + -inf
-        // 2. the topk_group best groups, one shuffle argmax each; 3. their entries
-        bool taken = false;
-        for (int j = 0; j < a.topk_group; ++j) {
-            const bool cand = owner && !taken;
-            float bs = score;
-            int bg = cand ? lane : 64;          // 64: no candidate
+        // 2. the topk_group best groups: each group's rank = groups ahead of it
+        //    (32 independent shuffles, no chain of argmax rounds); 3. the kept
+        //    groups (rank < topk_group) write their entries
+        int grank = 0;
+#pragma unroll 8
+        for (int o = 0; o < 32; ++o) {
+            const float os = __shfl_sync(0xffffffffu, score, o);
+            if (o < a.n_group && ahead(os, o, score, lane)) ++grank;
+        }
+        if (owner && grank < a.topk_group) {
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-                const int og = __shfl_xor_sync(0xffffffffu, bg, o);
-                if (og < 64 && (bg == 64 || ahead(os, og, bs, bg))) {
-                    bs = os;
-                    bg = og;
-                }
-            }
-            if (lane == bg) {
-                taken = true;
-#pragma unroll
-                for (int i = 0; i < P; ++i) {
-                    s_v[warp][j * P + i] = v[i];
-                    s_e[warp][j * P + i] = id[i];
-                }
+            for (int i = 0; i < P; ++i) {
+                s_v[warp][grank * P + i] = v[i];
+                s_e[warp][grank * P + i] = id[i];
             }
         }
         __syncwarp();

@@ -377,8 +377,12 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
         for (int j = 0; j < UPT; ++j) {
             const int u = u0 + j * blockDim.x + tid;
             if (u < U) {
-                r[j][0] = ld_nc_v4(xr + 2 * u);
-                r[j][1] = ld_nc_v4(xr + 2 * u + 1);
+                if (a.x32) {
+                    ld_nc_v8(xr + 2 * u, r[j][0], r[j][1]);
+                } else {
+                    r[j][0] = ld_nc_v4(xr + 2 * u);
+                    r[j][1] = ld_nc_v4(xr + 2 * u + 1);
+                }
             } else {
                 r[j][0] = r[j][1] = make_uint4(0, 0, 0, 0);
             }
@@ -488,8 +492,12 @@ __global__ void __launch_bounds__(1024) k_pack_token(PackArgs a) {
             for (int j = 0; j < UPT; ++j) {
                 const int u = j * blockDim.x + tid;
                 if (u < U) {
-                    raw[j][0] = ld_nc_v4(xr + 2 * u);
-                    raw[j][1] = ld_nc_v4(xr + 2 * u + 1);
+                    if (a.x32) {
+                        ld_nc_v8(xr + 2 * u, raw[j][0], raw[j][1]);
+                    } else {
+                        raw[j][0] = ld_nc_v4(xr + 2 * u);
+                        raw[j][1] = ld_nc_v4(xr + 2 * u + 1);
+                    }
                 } else {
                     raw[j][0] = raw[j][1] = make_uint4(0, 0, 0, 0);
                 }

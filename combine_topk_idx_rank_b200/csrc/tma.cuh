@@ -13,7 +13,7 @@
 #define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
 #endif
 #ifndef EP_PACK_CODE_STORE
-#define EP_PACK_CODE_STORE 0   // quantised code stores: 0 default, 1 .cs, 2 L2 evict-first hint, 3 .wt
+#define EP_PACK_CODE_STORE 2   // quantised code stores: 0 default, 1 .cs, 2 L2 evict-first hint (measured best), 3 .wt
 #endif
 
 namespace ep {
