@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libep.so")
 OBJDIR = os.path.join(HERE, "_build")
-SOURCES = ["routing.cu", "pack.cu", "combine.cu", "gating.cu", "padding.cu", "ep_api.cu", "ep_noalloc.cu"]
+SOURCES = ["routing.cu", "pack.cu", "combine.cu", "gating.cu", "padding.cu", "peer.cu", "ep_api.cu", "ep_noalloc.cu"]
 HEADERS = ["ep_internal.cuh", "quant.cuh", "tma.cuh", os.path.join("..", "..", "include", "ep.h"),
            os.path.join("..", "..", "include", "ep_testing.h")]
 

@@ -1,7 +1,9 @@
 // C ABI of libep.so (declared in include/ep.h): argument validation,
 // workspace carving and the launch sequence of each call.  Stateless: every
 // buffer belongs to the caller, nothing is allocated here.
+#include <cuda.h>   // CUdeviceptr / CUresult types; driver calls are resolved at run time
 #include <stdio.h>
+#include <string.h>
 
 #include "ep_internal.cuh"
 #include "../../include/ep_testing.h"
@@ -426,6 +428,143 @@ ep_status_t ep_write_padding_rows(const int32_t* psum, const int32_t* counts, in
     p.recv_topk_idx = recv_topk_idx; p.recv_topk_weights = recv_topk_weights; p.K = K;
     p.recv_meta = recv_src_metadata; p.capacity = capacity;
     return cuda_status(launch_padding(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_route(const int64_t* topk_idx, const float* topk_weights, int32_t T, int32_t K, int32_t E, int32_t R,
+                     int32_t A, int32_t token_offset, int32_t* recv_topk_idx, float* recv_topk_weights,
+                     int64_t recv_capacity, ep_handle_t* h, void* ws, size_t ws_bytes, void* stream) {
+    if (!sizes_ok(T, K, E, R) || h == nullptr || A < 1) return EP_ERR_INVALID_ARG;
+    if (ep_recv_capacity_bound(T, K, E, A) >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
+    if (recv_capacity < 0 || recv_capacity >= (int64_t)INT32_MAX) return EP_ERR_INVALID_ARG;
+    if (h->psum_num_recv_tokens_per_expert == nullptr || h->num_recv_tokens_per_expert == nullptr ||
+        h->err == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (h->dst_buffer_slot_idx == nullptr || topk_idx == nullptr || topk_weights == nullptr))
+        return EP_ERR_INVALID_ARG;
+    if (recv_capacity > 0 && (h->recv_src_metadata == nullptr || recv_topk_idx == nullptr ||
+                              recv_topk_weights == nullptr))
+        return EP_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, K, E, R);
+    if (ws == nullptr || ws_bytes < L.total) return EP_ERR_INVALID_ARG;
+    h->num_tokens = T; h->num_topk = K; h->num_experts = E; h->num_ranks = R;
+    h->expert_alignment = A; h->num_rounds = 1; h->recv_capacity = recv_capacity; h->low_latency = 0;
+    RouteArgs r = route_args(ws, L, topk_idx, topk_weights, T, K, E, R);
+    r.A = A;
+    r.capacity = recv_capacity;
+    r.check_capacity = 1;
+    r.assign = 1;
+    r.vector_ok = aligned16(topk_idx) && aligned16(topk_weights) && aligned16(recv_topk_idx) &&
+                  aligned16(recv_topk_weights);
+    r.dst_slot = h->dst_buffer_slot_idx;
+    r.topk_copy = h->topk_idx;
+    r.recv_meta = h->recv_src_metadata;
+    r.recv_topk_idx = recv_topk_idx;
+    r.recv_topk_weights = recv_topk_weights;
+    r.psum = h->psum_num_recv_tokens_per_expert;
+    r.num_recv = h->num_recv_tokens_per_expert;
+    r.err_out = h->err;
+    r.token_offset = token_offset;
+    return cuda_status(launch_route(r, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_pack_peer(const void* x, const ep_handle_t* h, const int32_t* send_topk_idx,
+                         const float* send_topk_weights, const int32_t* counts_all, int32_t G, int32_t g, int32_t A,
+                         const ep_dispatch_opts_t* opts, void* const* peer_recv_x, void* const* peer_recv_scales,
+                         int32_t* const* peer_recv_topk_idx, float* const* peer_recv_topk_weights,
+                         int32_t* const* peer_recv_metadata, int64_t peer_capacity, void* stream) {
+    if (h == nullptr || opts == nullptr || counts_all == nullptr) return EP_ERR_INVALID_ARG;
+    const int T = h->num_tokens, K = h->num_topk, E = h->num_experts, H = h->hidden;
+    if (!sizes_ok(T, K, E, h->num_ranks) || G < 1 || g < 0 || g >= G || E % G != 0 || A < 1) return EP_ERR_INVALID_ARG;
+    if (H < 16 || H > 65536 || H % 16 != 0 || peer_capacity < 0) return EP_ERR_INVALID_ARG;
+    if (h->expert_alignment != 1 || h->topk_idx == nullptr || h->err == nullptr) return EP_ERR_INVALID_ARG;
+    const int quant = opts->quant;
+    const int qs = quant == EP_QUANT_NONE ? 16 : opts->quant_size;
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3 && quant != EP_QUANT_INT8) return EP_ERR_INVALID_ARG;
+    if (quant != EP_QUANT_NONE && !(qs == 16 || qs == 32 || qs == 64 || qs == 128 || qs == 256 || qs == 512))
+        return EP_ERR_INVALID_ARG;
+    if (quant != EP_QUANT_NONE && (H % qs != 0 || peer_recv_scales == nullptr)) return EP_ERR_INVALID_ARG;
+    if (opts->scale_ue8m0 && quant != EP_QUANT_NONE && !opts->round_scale) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || !aligned16(x) || h->dst_buffer_slot_idx == nullptr || send_topk_idx == nullptr ||
+                  send_topk_weights == nullptr || h->recv_src_metadata == nullptr))
+        return EP_ERR_INVALID_ARG;
+    if (peer_recv_x == nullptr || peer_recv_topk_idx == nullptr || peer_recv_topk_weights == nullptr ||
+        peer_recv_metadata == nullptr)
+        return EP_ERR_INVALID_ARG;
+    PeerPackArgs p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.T = T; p.H = H; p.K = K; p.E = E; p.G = G; p.g = g; p.A = A;
+    p.dst_slot = h->dst_buffer_slot_idx; p.topk_copy = h->topk_idx;
+    p.send_topk_idx = send_topk_idx; p.send_topk_weights = send_topk_weights; p.send_meta = h->recv_src_metadata;
+    p.counts_all = counts_all;
+    p.peer_x = peer_recv_x; p.peer_scales = peer_recv_scales; p.peer_topk_idx = peer_recv_topk_idx;
+    p.peer_topk_weights = peer_recv_topk_weights; p.peer_meta = peer_recv_metadata;
+    p.capacity = peer_capacity;
+    p.quant_size = qs; p.round_scale = opts->round_scale ? 1 : 0;
+    p.scale_bytes = (quant != EP_QUANT_NONE && opts->scale_ue8m0) ? 1 : 0;
+    p.err = h->err;
+    return cuda_status(launch_pack_peer(p, quant, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_receiver_layout(const int32_t* counts_all, int32_t G, int32_t g, int32_t E, int32_t A, int32_t* psum,
+                               int32_t* counts, void* stream) {
+    if (counts_all == nullptr || psum == nullptr || counts == nullptr) return EP_ERR_INVALID_ARG;
+    if (G < 1 || g < 0 || g >= G || E < 1 || E > kMaxExperts || E % G != 0 || A < 1) return EP_ERR_INVALID_ARG;
+    return cuda_status(launch_receiver_layout(counts_all, G, g, E, A, psum, counts, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_combine_peer(void* const* peer_y, const ep_handle_t* h, const int32_t* counts_all, int32_t G, int32_t g,
+                            int32_t A, const float* topk_weights, void* out, int64_t peer_capacity, void* stream) {
+    if (h == nullptr || counts_all == nullptr || peer_y == nullptr) return EP_ERR_INVALID_ARG;
+    const int T = h->num_tokens, K = h->num_topk, E = h->num_experts, H = h->hidden;
+    if (!sizes_ok(T, K, E, h->num_ranks) || G < 1 || g < 0 || g >= G || E % G != 0 || A < 1) return EP_ERR_INVALID_ARG;
+    if (H < 8 || H > 65536 || H % 8 != 0 || peer_capacity < 0 || h->err == nullptr) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (out == nullptr || !aligned16(out) || topk_weights == nullptr || h->dst_buffer_slot_idx == nullptr ||
+                  h->topk_idx == nullptr))
+        return EP_ERR_INVALID_ARG;
+    PeerCombineArgs c{};
+    c.peer_y = peer_y;
+    c.T = T; c.H = H; c.K = K; c.E = E; c.G = G; c.g = g; c.A = A;
+    c.dst_slot = h->dst_buffer_slot_idx; c.topk_copy = h->topk_idx; c.topk_weights = topk_weights;
+    c.counts_all = counts_all; c.out = static_cast<uint16_t*>(out); c.capacity = peer_capacity; c.err = h->err;
+    return cuda_status(launch_combine_peer(c, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_ipc_export(const void* ptr, void* handle64, int64_t* offset) {
+    if (ptr == nullptr || handle64 == nullptr || offset == nullptr) return EP_ERR_INVALID_ARG;
+    static_assert(sizeof(cudaIpcMemHandle_t) == 64, "64-byte IPC handle");
+    // the allocation's base (allocators hand out pieces of larger allocations):
+    // cuMemGetAddressRange, resolved through the runtime
+    typedef CUresult (*RangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+    static RangeFn range = nullptr;
+    if (range == nullptr) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || f == nullptr)
+            return EP_ERR_CUDA;
+        range = reinterpret_cast<RangeFn>(f);
+    }
+    CUdeviceptr base = 0;
+    size_t bytes = 0;
+    if (range(&base, &bytes, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return EP_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    ep_status_t s = cuda_status(cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)));
+    if (s) return s;
+    memcpy(handle64, &h, sizeof h);
+    *offset = (int64_t)(reinterpret_cast<uintptr_t>(ptr) - (uintptr_t)base);
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_import(const void* handle64, void** base) {
+    if (handle64 == nullptr || base == nullptr) return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle64, sizeof h);
+    return cuda_status(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+ep_status_t ep_ipc_close(void* base) {
+    if (base == nullptr) return EP_ERR_INVALID_ARG;
+    return cuda_status(cudaIpcCloseMemHandle(base));
 }
 
 ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status) {

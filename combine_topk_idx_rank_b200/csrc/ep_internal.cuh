@@ -163,12 +163,48 @@ struct PadArgs {
     int64_t capacity;
 };
 
+// Multi-GPU pack and combine through peer memory (peer.cu).
+struct PeerPackArgs {
+    const uint16_t* x;          // this GPU's tokens [T, H]
+    int T, H, K, E, G, g, A;
+    const int32_t* dst_slot;    // [T, K] send rows (routing with alignment 1)
+    const int32_t* topk_copy;   // [T, K] expert ids (-1 = masked)
+    const int32_t* send_topk_idx;      // [rows, K] per send row
+    const float* send_topk_weights;    // [rows, K]
+    const int32_t* send_meta;          // [rows, 2]
+    const int32_t* counts_all;  // [G, E]
+    void* const* peer_x;        // [G] receivers' recv_x
+    void* const* peer_scales;   // [G] or null (bf16)
+    int32_t* const* peer_topk_idx;
+    float* const* peer_topk_weights;
+    int32_t* const* peer_meta;
+    int64_t capacity;           // rows of every receiver's layout
+    int quant_size, round_scale, scale_bytes;
+    int32_t* err;
+};
+
+struct PeerCombineArgs {
+    void* const* peer_y;        // [G] receivers' expert outputs (bf16)
+    int T, H, K, E, G, g, A;
+    const int32_t* dst_slot;
+    const int32_t* topk_copy;
+    const float* topk_weights;
+    const int32_t* counts_all;
+    uint16_t* out;
+    int64_t capacity;
+    int32_t* err;
+};
+
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_pack(const PackArgs& a, int quant, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t st);
 cudaError_t launch_padding(const PadArgs& a, cudaStream_t st);
+cudaError_t launch_pack_peer(const PeerPackArgs& a, int quant, cudaStream_t st);
+cudaError_t launch_combine_peer(const PeerCombineArgs& a, cudaStream_t st);
+cudaError_t launch_receiver_layout(const int32_t* C, int G, int g, int E, int A, int32_t* psum, int32_t* counts,
+                                   cudaStream_t st);
 
 int device_sm_count();
 

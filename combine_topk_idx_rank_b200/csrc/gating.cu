@@ -16,11 +16,11 @@
 //
 // One warp per token.  Lane g owns group g: it streams the group's S logits
 // (16-byte loads when S % 4 == 0) through a sorted per_group-entry insertion
-// list, then sums the list for the group's score.  Each lane counts the groups
-// ahead of its own (one shuffle per group, all independent); the lanes of the
-// topk_group best groups write their entries to shared memory, and lanes
-// 0..K-1 each take one entry, count the entries ahead of it (its output
-// position), and compute its weight.
+// list, then sums the list for the group's score.  The topk_group best groups
+// are taken one at a time by a warp max-reduction of order-preserving keys of
+// the scores (ties: the lowest lane, i.e. the lower group id); their lanes
+// write their entries to shared memory, and lanes 0..K-1 each take one entry,
+// count the entries ahead of it (its output position), and compute its weight.
 // Non-finite logits set EP_ERR_NONFINITE; they are then ordered as -inf (NaN)
 // or +-inf so that the outputs stay K distinct in-range ids.
 #include <math.h>
@@ -37,6 +37,13 @@ constexpr int kGateWarps = 8;   // tokens per CTA
 
 // True if (v, e) ranks ahead of (w, f): larger value, then lower id.
 __device__ __forceinline__ bool ahead(float v, int e, float w, int f) { return v > w || (v == w && e < f); }
+
+// An unsigned key with the order of the (non-NaN) floats, -0 and +0 equal:
+// every key is above 0, which the group selection uses for "no candidate".
+__device__ __forceinline__ uint32_t order_key(float x) {
+    const uint32_t u = __float_as_uint(x == 0.0f ? 0.0f : x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 __device__ __forceinline__ float sanitize(float x, int& bad) {
     if (!isfinite(x)) bad = 1;
@@ -114,20 +121,22 @@ __global__ void __launch_bounds__(kGateWarps * 32) k_gate(GateArgs a) {
 #pragma unroll
         for (int j = 1; j < P; ++j) score = score + v[j];
         if (score != score) score = -INFINITY;   // +inf + -inf
-        // 2. the topk_group best groups: each group's rank = groups ahead of it
-        //    (32 independent shuffles, no chain of argmax rounds); 3. the kept
-        //    groups (rank < topk_group) write their entries
-        int grank = 0;
-#pragma unroll 8
-        for (int o = 0; o < 32; ++o) {
-            const float os = __shfl_sync(0xffffffffu, score, o);
-            if (o < a.n_group && ahead(os, o, score, lane)) ++grank;
-        }
-        if (owner && grank < a.topk_group) {
+        // 2. the topk_group best groups, one warp max-reduction each: the
+        //    largest score's order key, then the lowest lane holding it (equal
+        //    scores: the lower group id); 3. the kept groups write their entries
+        bool taken = false;
+        const uint32_t key = order_key(score);
+        for (int j = 0; j < a.topk_group; ++j) {
+            const bool cand = owner && !taken;
+            const uint32_t best = __reduce_max_sync(0xffffffffu, cand ? key : 0u);
+            const int win = __ffs(__ballot_sync(0xffffffffu, cand && key == best)) - 1;
+            if (lane == win) {
+                taken = true;
 #pragma unroll
-            for (int i = 0; i < P; ++i) {
-                s_v[warp][grank * P + i] = v[i];
-                s_e[warp][grank * P + i] = id[i];
+                for (int i = 0; i < P; ++i) {
+                    s_v[warp][j * P + i] = v[i];
+                    s_e[warp][j * P + i] = id[i];
+                }
             }
         }
         __syncwarp();

@@ -36,7 +36,8 @@ _QUANT = {None: 0, "none": 0, "fp8": 1, "int8": 2, "mxfp4": 3}
 EXPORTED = ("ep_recv_capacity_bound", "ep_workspace_bytes", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_read_error", "ep_copy_recv_counts", "ep_status_string", "ep_dispatch_noalloc",
             "ep_dispatch_cached", "ep_dispatch_low_latency", "ep_combine_ex", "ep_group_limited_gating",
-            "ep_write_padding_rows")
+            "ep_write_padding_rows", "ep_route", "ep_pack_peer", "ep_receiver_layout", "ep_combine_peer",
+            "ep_ipc_export", "ep_ipc_import", "ep_ipc_close")
 
 
 class EPError(RuntimeError):
@@ -93,6 +94,20 @@ def _load(path: str = _LIB_PATH):
     L.ep_group_limited_gating.restype = C.c_int
     L.ep_write_padding_rows.argtypes = [p, p, i32, p, i64, p, i64, p, p, i32, p, i64, p]
     L.ep_write_padding_rows.restype = C.c_int
+    L.ep_route.argtypes = [p, p, i32, i32, i32, i32, i32, i32, p, p, i64, C.POINTER(_Handle), p, sz, p]
+    L.ep_route.restype = C.c_int
+    L.ep_pack_peer.argtypes = [p, C.POINTER(_Handle), p, p, p, i32, i32, i32, C.POINTER(_Opts), p, p, p, p, p, i64, p]
+    L.ep_pack_peer.restype = C.c_int
+    L.ep_receiver_layout.argtypes = [p, i32, i32, i32, i32, p, p, p]
+    L.ep_receiver_layout.restype = C.c_int
+    L.ep_combine_peer.argtypes = [p, C.POINTER(_Handle), p, i32, i32, i32, p, p, i64, p]
+    L.ep_combine_peer.restype = C.c_int
+    L.ep_ipc_export.argtypes = [p, p, C.POINTER(i64)]
+    L.ep_ipc_export.restype = C.c_int
+    L.ep_ipc_import.argtypes = [p, C.POINTER(p)]
+    L.ep_ipc_import.restype = C.c_int
+    L.ep_ipc_close.argtypes = [p]
+    L.ep_ipc_close.restype = C.c_int
     L.ep_status_string.argtypes = [C.c_int]
     L.ep_status_string.restype = C.c_char_p
     return L
@@ -533,3 +548,98 @@ def ep_write_padding_rows(psum: torch.Tensor, counts: torch.Tensor, recv_x: torc
                                     _ptr(recv_scales), srb, _ptr(recv_topk_idx), _ptr(recv_topk_weights), K,
                                     _ptr(recv_src_metadata), cap, _stream(recv_x.device))
     _check(st, "ep_write_padding_rows")
+
+
+# ----------------------------------------------- multi-GPU through peer memory
+
+@_on_tensor_device
+def ep_route(topk_idx: torch.Tensor, topk_weights: torch.Tensor, num_experts: int, num_ranks: int, hidden: int,
+             expert_alignment: int = 1, token_offset: int = 0, recv_capacity: Optional[int] = None):
+    """Routing without the pack (ep_dispatch's handle, recv_topk_idx / weights
+    and metadata): (recv_topk_idx, recv_topk_weights, handle)."""
+    _need_cuda(topk_idx, "topk_idx", torch.int64)
+    _need_cuda(topk_weights, "topk_weights", torch.float32)
+    T, K = topk_idx.shape
+    E, R, A = num_experts, num_ranks, expert_alignment
+    dev = topk_idx.device
+    cap = recv_capacity_bound(T, K, E, A) if recv_capacity is None else int(recv_capacity)
+    i32 = dict(dtype=torch.int32, device=dev)
+    h = EPHandle(T, K, E, R, hidden, A, 1, cap, torch.empty((T, K), **i32), torch.empty((E,), **i32),
+                 torch.empty((E,), **i32), torch.empty((max(cap, 1), 2), **i32), torch.empty((T, K), **i32),
+                 torch.zeros((1,), **i32))
+    rti = torch.empty((max(cap, 1), K), **i32)
+    rtw = torch.empty((max(cap, 1), K), dtype=torch.float32, device=dev)
+    ws = torch.empty((max(workspace_bytes(T, K, E, R), 256),), dtype=torch.uint8, device=dev)
+    ch = h._c()
+    st = _lib.ep_route(_ptr(topk_idx), _ptr(topk_weights), T, K, E, R, A, int(token_offset), _ptr(rti), _ptr(rtw),
+                       cap, C.byref(ch), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ep_route")
+    h.workspace_keepalive = ws
+    return rti, rtw, h
+
+
+def pointer_table(tensors, device) -> torch.Tensor:
+    """A device array of the given tensors' (or raw addresses') data pointers."""
+    addrs = [t if isinstance(t, int) else (0 if t is None else t.data_ptr()) for t in tensors]
+    return torch.tensor(addrs, dtype=torch.int64, device=device)
+
+
+@_on_tensor_device
+def ep_pack_peer(x: torch.Tensor, handle: EPHandle, send_topk_idx: torch.Tensor, send_topk_weights: torch.Tensor,
+                 counts_all: torch.Tensor, G: int, g: int, expert_alignment: int, peer_recv_x: torch.Tensor,
+                 peer_recv_scales: Optional[torch.Tensor], peer_recv_topk_idx: torch.Tensor,
+                 peer_recv_topk_weights: torch.Tensor, peer_recv_metadata: torch.Tensor, peer_capacity: int,
+                 quant: Optional[str] = None, quant_size: int = 128, round_scale: bool = False,
+                 scale_ue8m0: bool = False):
+    """Stores this GPU's rows straight into the receivers' layouts (peer_* are
+    device pointer tables from pointer_table)."""
+    q = None if quant in (None, "none") else quant
+    opts = _Opts(1, _QUANT[q], quant_size if q else 0, int(bool(round_scale)), 1, int(bool(scale_ue8m0)),
+                 None, None, None, 0)
+    st = _lib.ep_pack_peer(_ptr(x), C.byref(handle._c()), _ptr(send_topk_idx), _ptr(send_topk_weights),
+                           _ptr(counts_all), G, g, expert_alignment, C.byref(opts), _ptr(peer_recv_x),
+                           _ptr(peer_recv_scales), _ptr(peer_recv_topk_idx), _ptr(peer_recv_topk_weights),
+                           _ptr(peer_recv_metadata), int(peer_capacity), _stream(x.device))
+    _check(st, "ep_pack_peer")
+
+
+@_on_tensor_device
+def ep_receiver_layout(counts_all: torch.Tensor, G: int, g: int, expert_alignment: int):
+    """(psum [E/G], counts [E/G]) of this GPU's receive layout."""
+    E = counts_all.shape[1]
+    dev = counts_all.device
+    psum = torch.empty((E // G,), dtype=torch.int32, device=dev)
+    cnt = torch.empty((E // G,), dtype=torch.int32, device=dev)
+    st = _lib.ep_receiver_layout(_ptr(counts_all), G, g, E, expert_alignment, _ptr(psum), _ptr(cnt), _stream(dev))
+    _check(st, "ep_receiver_layout")
+    return psum, cnt
+
+
+@_on_tensor_device
+def ep_combine_peer(peer_y: torch.Tensor, handle: EPHandle, counts_all: torch.Tensor, G: int, g: int,
+                    expert_alignment: int, topk_weights: torch.Tensor, peer_capacity: int,
+                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Each of this GPU's tokens reduced from its rows in the receivers' y."""
+    if out is None:
+        out = torch.empty((handle.num_tokens, handle.hidden), dtype=torch.bfloat16, device=topk_weights.device)
+    st = _lib.ep_combine_peer(_ptr(peer_y), C.byref(handle._c()), _ptr(counts_all), G, g, expert_alignment,
+                              _ptr(topk_weights), _ptr(out), int(peer_capacity), _stream(out.device))
+    _check(st, "ep_combine_peer")
+    return out
+
+
+def ipc_export(t: torch.Tensor):
+    """(64-byte handle, offset) of the allocation holding t, for another process."""
+    h = C.create_string_buffer(64)
+    off = C.c_int64(0)
+    with torch.cuda.device(t.device):
+        _check(_lib.ep_ipc_export(_ptr(t), h, C.byref(off)), "ep_ipc_export")
+    return bytes(h.raw), off.value
+
+
+def ipc_import(handle: bytes, offset: int, device) -> int:
+    """The address, in this process, of an exported allocation plus offset."""
+    base = C.c_void_p(0)
+    with torch.cuda.device(device):
+        _check(_lib.ep_ipc_import(C.create_string_buffer(handle, 64), C.byref(base)), "ep_ipc_import")
+    return base.value + offset

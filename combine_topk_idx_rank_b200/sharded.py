@@ -257,3 +257,126 @@ class ShardedEP:
         sends, recvs = combine_messages(handle.plan)
         exchange(self.group, self.g, self.E, [(y, ret)], sends, recvs)
         return self.ops.combine(ret, st, topk_weights)
+
+
+# ------------------------------------------------- peer-memory data plane
+
+class PeerShardedEP:
+    """The same split of one batch over G GPUs (one process per GPU), with the
+    rows moving through peer memory instead of messages: each GPU routes its
+    own tokens (``ep_route``), the per-expert counts are all-gathered into
+    device memory, and ``ep_pack_peer`` stores every row (bf16 or quantised
+    once) and its per-row metadata straight into its receiver's layout through
+    peer pointers; ``ep_combine_peer`` loads each token's rows from the
+    receivers' expert outputs and reduces them in k order.  No host reads the
+    counts on the way.
+
+    Every GPU allocates its receive layout (and its expert-output buffer ``y``)
+    at the worst-case capacity and maps the other GPUs' through CUDA IPC once.
+    Steps are ordered across processes by a collective on the stream (NCCL) or
+    by a device sync and a host barrier (other backends)."""
+
+    def __init__(self, num_experts: int, num_ranks: int, hidden: int, num_topk: int, tokens_per_gpu: int,
+                 expert_alignment: int = 1, quant: Optional[str] = None, quant_size: int = 128,
+                 round_scale: bool = False, scale_ue8m0: bool = False, group=None, device=None):
+        from . import ep
+        self.ep = ep
+        self.group = group
+        self.G, self.g = dist.get_world_size(group), dist.get_rank(group)
+        if num_experts % num_ranks or num_ranks % self.G:
+            raise ValueError("num_ranks must divide num_experts and be a multiple of the GPU count")
+        self.E, self.R, self.H, self.K, self.A = num_experts, num_ranks, hidden, num_topk, expert_alignment
+        self.Tg = tokens_per_gpu
+        self.quant = None if quant in (None, "none") else quant
+        self.quant_size, self.round_scale, self.scale_ue8m0 = quant_size, round_scale, scale_ue8m0
+        self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.nccl = dist.get_backend(group) == "nccl"
+        # every row of the batch could land on one GPU
+        self.cap = self.Tg * self.G * self.K + (self.E // self.G) * (self.A - 1)
+        rx, rs = ep._recv_tensors(self.cap, hidden, self.quant, quant_size, scale_ue8m0, self.dev)
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        self.recv_x, self.recv_scales = rx, rs
+        self.recv_topk_idx = torch.empty((self.cap, self.K), **i32)
+        self.recv_topk_weights = torch.empty((self.cap, self.K), dtype=torch.float32, device=self.dev)
+        self.recv_meta = torch.empty((self.cap, 2), **i32)
+        self.y = torch.empty((self.cap, hidden), dtype=torch.bfloat16, device=self.dev)
+        self._imported = []
+        bufs = [self.recv_x, self.recv_scales, self.recv_topk_idx, self.recv_topk_weights, self.recv_meta, self.y]
+        tables = [self._peer_addresses(b) for b in bufs]
+        (self.t_x, self.t_scales, self.t_topk_idx, self.t_topk_weights, self.t_meta, self.t_y) = [
+            ep.pointer_table(t, self.dev) for t in tables]
+        self._flag = torch.zeros((1,), **i32)
+
+    def _peer_addresses(self, t):
+        """Every GPU's address of the same buffer, in this process."""
+        if t is None:
+            return [0] * self.G
+        torch.cuda.synchronize(self.dev)
+        mine = self.ep.ipc_export(t) if self.G > 1 else (b"", 0)
+        allh = [None] * self.G
+        dist.all_gather_object(allh, mine, group=self.group)
+        out = []
+        for q, (h, off) in enumerate(allh):
+            if q == self.g:
+                out.append(t.data_ptr())
+            else:
+                addr = self.ep.ipc_import(h, off, self.dev)
+                self._imported.append(addr - off)
+                out.append(addr)
+        return out
+
+    def _order(self):
+        """Every GPU has finished the work it queued before this point."""
+        if self.nccl:
+            dist.all_reduce(self._flag, group=self.group)
+        else:
+            torch.cuda.synchronize(self.dev)
+            dist.barrier(group=self.group)
+
+    def _gather_counts(self, counts):
+        if self.nccl:
+            out = torch.empty((self.G, self.E), dtype=torch.int32, device=self.dev)
+            dist.all_gather_into_tensor(out, counts, group=self.group)
+            return out
+        parts = [torch.empty((self.E,), dtype=torch.int32) for _ in range(self.G)]
+        dist.all_gather(parts, counts.cpu(), group=self.group)
+        return torch.stack(parts).to(self.dev)
+
+    def dispatch(self, x, topk_idx, topk_weights):
+        """This GPU's tokens -> (recv_x, recv_scales, recv_topk_idx,
+        recv_topk_weights, handle) of its experts (views of its layout)."""
+        ep = self.ep
+        rti, rtw, h = ep.ep_route(topk_idx, topk_weights, self.E, self.R, self.H, 1, token_offset=self.g * self.Tg)
+        counts_all = self._gather_counts(h.num_recv_tokens_per_expert)
+        self._order()                     # the receivers are done with their previous rows
+        ep.ep_pack_peer(x, h, rti, rtw, counts_all, self.G, self.g, self.A, self.t_x, self.t_scales,
+                        self.t_topk_idx, self.t_topk_weights, self.t_meta, self.cap, self.quant, self.quant_size,
+                        self.round_scale, self.scale_ue8m0)
+        self._order()                     # every GPU's rows have landed
+        psum, cnt = ep.ep_receiver_layout(counts_all, self.G, self.g, self.A)
+        rows = int(psum[-1].item()) if psum.numel() else 0
+        ep.ep_write_padding_rows(psum, cnt, self.recv_x[:rows],
+                                 None if self.recv_scales is None else self.recv_scales[:rows],
+                                 self.recv_topk_idx[:rows], self.recv_topk_weights[:rows], self.recv_meta[:rows])
+        handle = dict(route=h, counts_all=counts_all, psum=psum, counts=cnt, rows=rows)
+        rs = None if self.recv_scales is None else self.recv_scales[:rows]
+        return self.recv_x[:rows], rs, self.recv_topk_idx[:rows], self.recv_topk_weights[:rows], handle
+
+    def combine(self, handle, topk_weights):
+        """After the experts wrote this GPU's outputs into ``self.y`` (received
+        order): this GPU's tokens, combined."""
+        self._order()                     # every receiver's y is written
+        out = self.ep.ep_combine_peer(self.t_y, handle["route"], handle["counts_all"], self.G, self.g, self.A,
+                                      topk_weights, self.cap)
+        self._order()                     # no receiver overwrites y while it is read
+        return out
+
+    def close(self):
+        for base in self._imported:
+            self.ep._lib.ep_ipc_close(C_void_p(base))
+        self._imported = []
+
+
+def C_void_p(v):
+    import ctypes
+    return ctypes.c_void_p(v)

@@ -334,6 +334,82 @@ ep_status_t ep_write_padding_rows(const int32_t* psum, const int32_t* counts, in
                                   int32_t* recv_topk_idx, float* recv_topk_weights, int32_t K,
                                   int32_t* recv_src_metadata, int64_t capacity, void* stream);
 
+/*
+ * Expert parallelism over G GPUs through peer memory (one process per GPU,
+ * NVLink / NVSwitch peer loads and stores; comparative analysis section 6.1,
+ * the normal mode's dispatch of each rank's tokens into the receivers'
+ * buffers, and section 9.2, combine).  GPU g of G holds the logical ranks
+ * [g R/G, (g+1) R/G): tokens [g T/G, (g+1) T/G) of the batch and experts
+ * [g E/G, (g+1) E/G).  Each GPU ends with the single-GPU result restricted to
+ * itself (its experts' rows in (expert, token, k) order, padded to the
+ * alignment A; its own tokens combined).
+ *   1. ep_route on every GPU: routing of its own tokens with alignment 1 (its
+ *      send order); handle->num_recv_tokens_per_expert is its row of the
+ *      count matrix C [G, E];
+ *   2. the caller all-gathers C into device memory on every GPU (NCCL);
+ *   3. ep_pack_peer on every GPU: each entry's row on its receiver
+ *      d = e / (E/G) is computed from C on the device, and the row (bf16 or
+ *      quantised), its scales, recv_topk_idx / weights and metadata are stored
+ *      straight into d's layout through the peer pointer tables;
+ *   4. the caller orders the GPUs (a collective after the packs); each
+ *      receiver runs ep_receiver_layout and ep_write_padding_rows;
+ *   5. after the experts, ep_combine_peer on every GPU loads each of its
+ *      tokens' rows from the receivers' y through peer pointers and reduces
+ *      them in k order.
+ * Peer pointer tables are device arrays of G pointers (entry g' = that
+ * buffer on GPU g', mapped into this process; entry g = this GPU's own).
+ * Nothing here waits on another GPU: the caller's collectives order the
+ * steps.  No TMA or bulk load with cluster multicast is used.
+ */
+
+/* Routing only (steps 1): ep_dispatch's handle, recv_topk_idx,
+ * recv_topk_weights and metadata, in the same layout and with the same
+ * arguments (token_offset included), but no rows: the rows are packed by
+ * ep_pack_peer.  recv_capacity >= rows needed with this alignment. */
+ep_status_t ep_route(const int64_t* topk_idx, const float* topk_weights, int32_t T, int32_t K, int32_t E,
+                     int32_t R, int32_t expert_alignment, int32_t token_offset, int32_t* recv_topk_idx,
+                     float* recv_topk_weights, int64_t recv_capacity, ep_handle_t* handle, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Step 3.  x: this GPU's tokens [T, H]; handle from ep_route (alignment 1);
+ * send_topk_idx / send_topk_weights: the recv_topk_* arrays ep_route wrote
+ * (rows in send order); counts_all: device int32 [G, E]; opts: quant,
+ * quant_size, round_scale and scale_ue8m0 as in ep_dispatch (FP8 / int8
+ * groups of 16..512 channels, or none); A: the receivers' expert alignment;
+ * peer_*: device arrays of G pointers to the receivers' recv_x, recv_scales
+ * (may be NULL for bf16), recv_topk_idx, recv_topk_weights and
+ * recv_src_metadata, each with peer_capacity rows.  Rows at or past
+ * peer_capacity are not written (EP_ERR_CAPACITY in handle->err). */
+ep_status_t ep_pack_peer(const void* x, const ep_handle_t* handle, const int32_t* send_topk_idx,
+                         const float* send_topk_weights, const int32_t* counts_all, int32_t G, int32_t g,
+                         int32_t A, const ep_dispatch_opts_t* opts, void* const* peer_recv_x,
+                         void* const* peer_recv_scales, int32_t* const* peer_recv_topk_idx,
+                         float* const* peer_recv_topk_weights, int32_t* const* peer_recv_metadata,
+                         int64_t peer_capacity, void* stream);
+
+/* Step 4: this GPU's receive layout from counts_all: psum [E/G] (inclusive
+ * prefix of the aligned totals over its experts) and counts [E/G]. */
+ep_status_t ep_receiver_layout(const int32_t* counts_all, int32_t G, int32_t g, int32_t E, int32_t A,
+                               int32_t* psum, int32_t* counts, void* stream);
+
+/* Step 5: for each of this GPU's tokens t, out[t] = bf16_rne(fma chain in k
+ * order of topk_weights[t,k] * y_d[row]) over the unmasked entries, where
+ * row on receiver d is the one ep_pack_peer wrote; peer_y: device array of G
+ * pointers to the receivers' expert outputs (bf16, peer_capacity rows). */
+ep_status_t ep_combine_peer(void* const* peer_y, const ep_handle_t* handle, const int32_t* counts_all, int32_t G,
+                            int32_t g, int32_t A, const float* topk_weights, void* out, int64_t peer_capacity,
+                            void* stream);
+
+/* CUDA IPC for the peer pointer tables.  ep_ipc_export writes the 64-byte IPC
+ * handle of the device allocation that holds ptr to handle64 and ptr's offset
+ * inside that allocation to *offset; ep_ipc_import opens such a handle in
+ * another process of the same machine (on the current device) and returns
+ * the allocation's address there (add the offset); ep_ipc_close releases an
+ * imported address.  Host calls; they allocate nothing on the device. */
+ep_status_t ep_ipc_export(const void* ptr, void* handle64, int64_t* offset);
+ep_status_t ep_ipc_import(const void* handle64, void** base);
+ep_status_t ep_ipc_close(void* base);
+
 /* Waits for `stream`, then copies the device status word to *host_status.
  * Returns EP_OK, or EP_ERR_CUDA if the wait or the copy failed. */
 ep_status_t ep_read_error(const int32_t* err, void* stream, int32_t* host_status);
