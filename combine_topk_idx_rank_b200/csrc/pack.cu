@@ -45,21 +45,12 @@ namespace {
 
 constexpr int kBulkChunk = 16384;          // max bytes per pipeline stage
 
-// 16 bytes of quantised codes to a received row.
-__device__ __forceinline__ void st_code_v4(void* p, uint4 v) {
-#if EP_PACK_CODE_STORE == 1
-    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-#elif EP_PACK_CODE_STORE == 2
+// 16 bytes of quantised codes to a received row, with the L2 policy `pol`
+// (evict-first: the row is read once, by the experts, long after).
+__device__ __forceinline__ void st_code_v4(void* p, uint4 v, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w), "l"(l2_evict_first())
+                 "r"(v.z), "r"(v.w), "l"(pol)
                  : "memory");
-#elif EP_PACK_CODE_STORE == 3
-    asm volatile("st.global.wt.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-#else
-    st_v4(p, v);
-#endif
 }
 
 // Padding map from the handle: expert e's padding rows are
@@ -333,7 +324,10 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 // item is one pass (UPT x blockDim units) over one token's row, or one padding
 // row.  The CTA's next item is fetched (its x units into registers, its
 // destination rows into the other half of s_slot) before the current item is
-// quantised and stored, so its loads are in flight during that work.
+// quantised and stored, so its loads are in flight during that work.  A
+// warp's units cover whole groups; the K x (groups of the warp) scale stores
+// of an item are spread over the warp's lanes, one or a few per lane, instead
+// of one lane of each group storing K scales.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_group(PackArgs a) {
     grid_dependency_wait();
@@ -342,9 +336,10 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
     __shared__ int s_slot[2][kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
+    constexpr int kGroupsPerWarp = 32 / kLanes;
     constexpr float kQmax = QUANT == kQuantFp8 ? 448.0f : 127.0f;
     constexpr int kUnitBytes = QUANT == kQuantMxfp4 ? 8 : 16;   // code bytes of 16 channels
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int U = a.H / 16;
     const int per_pass = UPT * blockDim.x;
     const int passes = (U + per_pass - 1) / per_pass;
@@ -428,20 +423,42 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
                     q[j] = quant16<QUANT>(f, sc[j]);
                 }
             }
+            // codes: per received row one 32 x 32 -> 64-bit multiply-add and
+            // one store per unit (a row is at most 64 KB of codes)
+            uint8_t* const xb = a.recv_x + (size_t)(u0 + tid) * kUnitBytes;
+            const int rb = (int)row_bytes;
             for (int k = 0; k < a.K; ++k) {
                 const int slot = s_slot[buf][k];
                 if (slot < 0) continue;
-                uint8_t* dst = a.recv_x + (size_t)slot * row_bytes;
+                uint8_t* const dst = xb + (long long)slot * rb;
 #pragma unroll
                 for (int j = 0; j < UPT; ++j) {
-                    const int u = u0 + j * blockDim.x + tid;
-                    if (u < U) {
+                    if (u0 + j * (int)blockDim.x + tid < U) {
+                        uint8_t* const p = dst + j * (int)blockDim.x * kUnitBytes;
                         if constexpr (QUANT == kQuantMxfp4) {
-                            *reinterpret_cast<uint2*>(dst + 8 * (size_t)u) = make_uint2(q[j].x, q[j].y);
+                            *reinterpret_cast<uint2*>(p) = make_uint2(q[j].x, q[j].y);
                         } else {
-                            st_code_v4(dst + 16 * (size_t)u, q[j]);
+                            st_code_v4(p, q[j], l2_evict_first());
                         }
-                        if ((u % kLanes) == 0) store_scale(a, (size_t)slot * nscales + u / kLanes, sc[j]);
+                    }
+                }
+            }
+            // scales: entry i of the warp's K x kGroupsPerWarp stores of pass
+            // slice j is (row i / kGroupsPerWarp, group i % kGroupsPerWarp of
+            // the warp); lane i % 32 stores it, with the scale of the group's
+            // first lane
+#pragma unroll
+            for (int j = 0; j < UPT; ++j) {
+                const int wu = u0 + j * (int)blockDim.x + (tid & ~31);   // the warp's first unit
+                const int n = a.K * kGroupsPerWarp;
+                for (int i0 = 0; i0 < n; i0 += 32) {
+                    const int i = i0 + lane;
+                    const int g = i % kGroupsPerWarp;
+                    const float s = __shfl_sync(0xffffffffu, sc[j], g * kLanes);
+                    const int ug = wu + g * kLanes;
+                    if (i < n && ug < U) {
+                        const int row = s_slot[buf][i / kGroupsPerWarp];
+                        if (row >= 0) store_scale(a, (size_t)row * nscales + ug / kLanes, s);
                     }
                 }
             }
@@ -577,15 +594,16 @@ cudaError_t launch_group(const PackArgs& a, cudaStream_t st) {
     if constexpr (QUANT == kQuantMxfp4) {
         if (a.quant_size != 32) return cudaErrorInvalidValue;
         return run(k_pack_group<kQuantMxfp4, 32, P>, threads, a, st);
-    }
-    switch (a.quant_size) {
-        case 16: return run(k_pack_group<QUANT, 16, P>, threads, a, st);
-        case 32: return run(k_pack_group<QUANT, 32, P>, threads, a, st);
-        case 64: return run(k_pack_group<QUANT, 64, P>, threads, a, st);
-        case 128: return run(k_pack_group<QUANT, 128, P>, threads, a, st);
-        case 256: return run(k_pack_group<QUANT, 256, P>, threads, a, st);
-        case 512: return run(k_pack_group<QUANT, 512, P>, threads, a, st);
-        default: return cudaErrorInvalidValue;
+    } else {
+        switch (a.quant_size) {
+            case 16: return run(k_pack_group<QUANT, 16, P>, threads, a, st);
+            case 32: return run(k_pack_group<QUANT, 32, P>, threads, a, st);
+            case 64: return run(k_pack_group<QUANT, 64, P>, threads, a, st);
+            case 128: return run(k_pack_group<QUANT, 128, P>, threads, a, st);
+            case 256: return run(k_pack_group<QUANT, 256, P>, threads, a, st);
+            case 512: return run(k_pack_group<QUANT, 512, P>, threads, a, st);
+            default: return cudaErrorInvalidValue;
+        }
     }
 }
 

@@ -12,9 +12,6 @@
 #ifndef EP_PACK_STORE_HINT
 #define EP_PACK_STORE_HINT 0   // 1: bulk stores of received rows carry an L2 evict-first policy
 #endif
-#ifndef EP_PACK_CODE_STORE
-#define EP_PACK_CODE_STORE 2   // quantised code stores: 0 default, 1 .cs, 2 L2 evict-first hint (measured best), 3 .wt
-#endif
 
 namespace ep {
 namespace {
@@ -52,14 +49,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
-#if EP_PACK_LOAD_HINT || EP_PACK_STORE_HINT || EP_PACK_CODE_STORE == 2
-// L2 policy that marks lines for early eviction (rows are read or written once)
+// L2 policy that marks lines for early eviction (rows are read or written
+// once)
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
-#endif
 __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
 #if EP_PACK_LOAD_HINT
     asm volatile(
