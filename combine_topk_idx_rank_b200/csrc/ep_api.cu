@@ -64,10 +64,12 @@ RouteArgs route_args(void* ws, const WsLayout& L, const int64_t* topk_idx, const
 // The pack kernel(s) of a dispatch: one launch per round, each a
 // programmatic dependent of the previous kernel on the stream.  Rows come
 // from handle->dst_buffer_slot_idx; the padding map from the handle's psum
-// and unaligned counts.
+// and unaligned counts.  `routed`: the routing kernel was launched just
+// before on the stream, so x was complete when it started and the packs may
+// read x before their dependency wait.
 ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R, int quant, int quant_size,
                                const ep_dispatch_opts_t* opts, void* recv_x, float* recv_scales,
-                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st) {
+                               int64_t recv_capacity, const ep_handle_t* h, cudaStream_t st, bool routed) {
     ep_status_t s;
     if (opts->event_pack_begin) {
         s = cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(opts->event_pack_begin), st));
@@ -90,6 +92,7 @@ ep_status_t launch_pack_rounds(const void* x, int T, int H, int K, int E, int R,
             pa.scale_bytes = (quant == EP_QUANT_MXFP4 || (quant != EP_QUANT_NONE && opts->scale_ue8m0)) ? 1 : 0;
             pa.err = h->err;
             pa.x32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;   // rows of H % 16 == 0 channels stay aligned
+            pa.early_x = routed ? 1 : 0;
             s = cuda_status(launch_pack(pa, quant, st));
             if (s) return s;
         }
@@ -226,7 +229,7 @@ ep_status_t dispatch_impl(const void* x, int32_t T, int32_t H, const int64_t* to
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, recv_capacity, h,
-                              st);
+                              st, true);
 }
 
 }  // namespace
@@ -327,7 +330,7 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t T, int32_t H, const i
     r.token_offset = opts->token_offset;
     ep_status_t s = cuda_status(launch_route(r, st));
     if (s) return s;
-    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st);
+    return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, rows, h, st, true);
 }
 
 ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dispatch_opts_t* opts,
@@ -349,7 +352,7 @@ ep_status_t ep_dispatch_cached(const void* x, const ep_handle_t* h, const ep_dis
     if (h->recv_capacity > 0 && recv_x == nullptr) return EP_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(recv_x)) return EP_ERR_INVALID_ARG;
     return launch_pack_rounds(x, T, H, K, E, R, quant, quant_size, opts, recv_x, recv_scales, h->recv_capacity, h,
-                              static_cast<cudaStream_t>(stream));
+                              static_cast<cudaStream_t>(stream), false);
 }
 
 ep_status_t ep_combine_ex(const void* y, const float* y_scales, int32_t y_quant, int32_t y_quant_size,

@@ -120,6 +120,8 @@ struct PackArgs {
     int quant_size, round_scale;
     int scale_bytes;            // scales stored as UE8M0 bytes (MXFP4 always)
     int x32;                    // x is 32-byte aligned: a 16-channel unit is one 32-byte load
+    int early_x;                // x was complete when the kernel before this one started (the
+                                // routing kernel precedes): x may be read before the wait
     int32_t* err;
 };
 

@@ -328,11 +328,11 @@ __global__ void __launch_bounds__(256) k_pack_bf16(PackArgs a) {
 // warp's units cover whole groups; the K x (groups of the warp) scale stores
 // of an item are spread over the warp's lanes, one or a few per lane, instead
 // of one lane of each group storing K scales.
+// With a.early_x (the routing kernel runs just before, so x was complete
+// before it started), the CTA's first item is loaded and quantised before the
+// wait for the routing results, while routing runs.
 template <int QUANT, int G, int UPT>
 __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_group(PackArgs a) {
-    grid_dependency_wait();
-    grid_launch_dependents();
-    if (routing_gave_up(a)) return;
     __shared__ int s_slot[2][kMaxTopk];
     __shared__ int s_pad_base[kMaxExperts + 1], s_pad_start[kMaxExperts], s_warp[32];
     constexpr int kLanes = G / 16;
@@ -345,9 +345,7 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
     const int passes = (U + per_pass - 1) / per_pass;
     const size_t row_bytes = (size_t)U * kUnitBytes;
     const int nscales = a.H / G;
-    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
     const int n_tok = a.n_tok_items * passes;
-    const int n_items = n_tok + n_pad;
 
     // item -> token, and the first unit of its pass; with one pass per row and
     // one round (every workload but the longest rows and rounds) the item is
@@ -363,8 +361,8 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
         u0 = (item - ti * passes) * per_pass;
         t = token_of_item(ti, a.tokens_per_rank, a.per_round, a.round);
     };
-    // issues the loads of a token item: its units into r, its rows into slot
-    auto fetch = [&](int item, uint4 (&r)[UPT][2], int& slot) {
+    // issues the loads of a token item's units into r
+    auto fetch_x = [&](int item, uint4 (&r)[UPT][2]) {
         int t, u0;
         locate(item, t, u0);
         const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
@@ -382,13 +380,105 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
                 r[j][0] = r[j][1] = make_uint4(0, 0, 0, 0);
             }
         }
-        slot = tid < a.K ? a.dst_slot[(int64_t)t * a.K + tid] : -1;
     };
+    // threads 0..K-1: the received row of entry tid of a token item
+    auto fetch_slot = [&](int item) {
+        int t, u0;
+        locate(item, t, u0);
+        return tid < a.K ? a.dst_slot[(int64_t)t * a.K + tid] : -1;
+    };
+    auto quantize = [&](const uint4 (&r)[UPT][2], uint4 (&q)[UPT], float (&sc)[UPT]) {
+#pragma unroll
+        for (int j = 0; j < UPT; ++j) {
+            float f[16];
+            unpack16(r[j][0], r[j][1], f);
+            float m = amax16(f);
+#pragma unroll
+            for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if constexpr (QUANT == kQuantMxfp4) {
+                sc[j] = mx_scale(m);
+                const uint2 c = quant16_fp4(f, sc[j]);
+                q[j] = make_uint4(c.x, c.y, 0, 0);
+            } else {
+                sc[j] = finish_scale(m, kQmax, a.round_scale);
+                q[j] = quant16<QUANT>(f, sc[j]);
+            }
+        }
+    };
+    // the codes and scales of a token item to its received rows s_slot[b]
+    auto store_item = [&](int item, const uint4 (&q)[UPT], const float (&sc)[UPT], int b) {
+        int t, u0;
+        locate(item, t, u0);
+        // codes: per received row one 32 x 32 -> 64-bit multiply-add and
+        // one store per unit (a row is at most 64 KB of codes)
+        uint8_t* const xb = a.recv_x + (size_t)(u0 + tid) * kUnitBytes;
+        const int rb = (int)row_bytes;
+        for (int k = 0; k < a.K; ++k) {
+            const int slot = s_slot[b][k];
+            if (slot < 0) continue;
+            uint8_t* const dst = xb + (long long)slot * rb;
+#pragma unroll
+            for (int j = 0; j < UPT; ++j) {
+                if (u0 + j * (int)blockDim.x + tid < U) {
+                    uint8_t* const p = dst + j * (int)blockDim.x * kUnitBytes;
+                    if constexpr (QUANT == kQuantMxfp4) {
+                        *reinterpret_cast<uint2*>(p) = make_uint2(q[j].x, q[j].y);
+                    } else {
+                        st_code_v4(p, q[j], l2_evict_first());
+                    }
+                }
+            }
+        }
+        // scales: entry i of the warp's K x kGroupsPerWarp stores of pass
+        // slice j is (row i / kGroupsPerWarp, group i % kGroupsPerWarp of
+        // the warp); lane i % 32 stores it, with the scale of the group's
+        // first lane
+#pragma unroll
+        for (int j = 0; j < UPT; ++j) {
+            const int wu = u0 + j * (int)blockDim.x + (tid & ~31);   // the warp's first unit
+            const int n = a.K * kGroupsPerWarp;
+            for (int i0 = 0; i0 < n; i0 += 32) {
+                const int i = i0 + lane;
+                const int g = i % kGroupsPerWarp;
+                const float s = __shfl_sync(0xffffffffu, sc[j], g * kLanes);
+                const int ug = wu + g * kLanes;
+                if (i < n && ug < U) {
+                    const int row = s_slot[b][i / kGroupsPerWarp];
+                    if (row >= 0) store_scale(a, (size_t)row * nscales + ug / kLanes, s);
+                }
+            }
+        }
+    };
+
+    int item = blockIdx.x;
+    const bool early = a.early_x != 0 && item < n_tok;
+    uint4 q0[UPT];
+    float sc0[UPT];
+    if (early) {
+        uint4 r0[UPT][2];
+        fetch_x(item, r0);
+        quantize(r0, q0, sc0);
+    }
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (routing_gave_up(a)) return;
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
+    const int n_items = n_tok + n_pad;
+    if (early) {
+        // the first item, quantised during routing: its rows, then its stores
+        const int slot = fetch_slot(item);
+        if (tid < a.K) s_slot[1][tid] = checked_row(a, slot);
+        __syncthreads();
+        store_item(item, q0, sc0, 1);
+        item += gridDim.x;
+    }
 
     uint4 raw[UPT][2];
     int slot_next = -1;
-    int item = blockIdx.x;
-    if (item < n_tok) fetch(item, raw, slot_next);
+    if (item < n_tok) {
+        fetch_x(item, raw);
+        slot_next = fetch_slot(item);
+    }
     if (tid < a.K) s_slot[0][tid] = checked_row(a, slot_next);
     __syncthreads();
     int buf = 0;
@@ -397,71 +487,17 @@ __global__ void __launch_bounds__(512 / UPT, EP_PACK_GROUP_MIN_BLOCKS) k_pack_gr
         uint4 nraw[UPT][2];
         slot_next = -1;
         if (nxt < n_tok) {
-            fetch(nxt, nraw, slot_next);
+            fetch_x(nxt, nraw);
+            slot_next = fetch_slot(nxt);
         } else {
 #pragma unroll
             for (int j = 0; j < UPT; ++j) nraw[j][0] = nraw[j][1] = make_uint4(0, 0, 0, 0);
         }
         if (item < n_tok) {
-            int t, u0;
-            locate(item, t, u0);
             uint4 q[UPT];
             float sc[UPT];
-#pragma unroll
-            for (int j = 0; j < UPT; ++j) {
-                float f[16];
-                unpack16(raw[j][0], raw[j][1], f);
-                float m = amax16(f);
-#pragma unroll
-                for (int o = kLanes / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if constexpr (QUANT == kQuantMxfp4) {
-                    sc[j] = mx_scale(m);
-                    const uint2 c = quant16_fp4(f, sc[j]);
-                    q[j] = make_uint4(c.x, c.y, 0, 0);
-                } else {
-                    sc[j] = finish_scale(m, kQmax, a.round_scale);
-                    q[j] = quant16<QUANT>(f, sc[j]);
-                }
-            }
-            // codes: per received row one 32 x 32 -> 64-bit multiply-add and
-            // one store per unit (a row is at most 64 KB of codes)
-            uint8_t* const xb = a.recv_x + (size_t)(u0 + tid) * kUnitBytes;
-            const int rb = (int)row_bytes;
-            for (int k = 0; k < a.K; ++k) {
-                const int slot = s_slot[buf][k];
-                if (slot < 0) continue;
-                uint8_t* const dst = xb + (long long)slot * rb;
-#pragma unroll
-                for (int j = 0; j < UPT; ++j) {
-                    if (u0 + j * (int)blockDim.x + tid < U) {
-                        uint8_t* const p = dst + j * (int)blockDim.x * kUnitBytes;
-                        if constexpr (QUANT == kQuantMxfp4) {
-                            *reinterpret_cast<uint2*>(p) = make_uint2(q[j].x, q[j].y);
-                        } else {
-                            st_code_v4(p, q[j], l2_evict_first());
-                        }
-                    }
-                }
-            }
-            // scales: entry i of the warp's K x kGroupsPerWarp stores of pass
-            // slice j is (row i / kGroupsPerWarp, group i % kGroupsPerWarp of
-            // the warp); lane i % 32 stores it, with the scale of the group's
-            // first lane
-#pragma unroll
-            for (int j = 0; j < UPT; ++j) {
-                const int wu = u0 + j * (int)blockDim.x + (tid & ~31);   // the warp's first unit
-                const int n = a.K * kGroupsPerWarp;
-                for (int i0 = 0; i0 < n; i0 += 32) {
-                    const int i = i0 + lane;
-                    const int g = i % kGroupsPerWarp;
-                    const float s = __shfl_sync(0xffffffffu, sc[j], g * kLanes);
-                    const int ug = wu + g * kLanes;
-                    if (i < n && ug < U) {
-                        const int row = s_slot[buf][i / kGroupsPerWarp];
-                        if (row >= 0) store_scale(a, (size_t)row * nscales + ug / kLanes, s);
-                    }
-                }
-            }
+            quantize(raw, q, sc);
+            store_item(item, q, sc, buf);
         } else {
             const int64_t row = pad_row(a.E, s_pad_base, s_pad_start, item - n_tok);
             if (row >= 0 && row < a.capacity) {
