@@ -104,6 +104,9 @@ struct RouteArgs {
     // > 0 only from the test entry points: raises the first grid barrier's
     // target past the number of CTAs, so that no CTA can pass it
     unsigned stall;
+    // 1: the per-chunk tables fit in shared memory; after the first barrier
+    // every CTA copies them in and sums the columns itself (no second phase)
+    int fold;
 };
 
 struct PackArgs {

@@ -12,7 +12,10 @@
 //      write the chunk's expert and rank histograms and is_token_in_rank;
 //   2. one warp per column of the [chunk, expert] histogram: exclusive prefix
 //      over the chunks (in place) and the column total = expert count;
-//      likewise the per-rank and error columns;
+//      likewise the per-rank and error columns.  When the tables fit in
+//      shared memory (a.fold) this phase and its barrier are skipped: every
+//      CTA copies the whole [chunk, expert] table in with cp.async and sums
+//      the columns it needs (expert totals, its chunk's prefix) itself;
 //   3. every CTA scans the aligned expert counts for the segment starts;
 //      row = segment start + chunk prefix + rank inside the chunk; write
 //      dst_buffer_slot_idx, recv_src_metadata, recv_topk_idx/weights and the
@@ -22,17 +25,32 @@
 // No sort, no global atomics except the barrier counter.
 #include "ep_internal.cuh"
 
+#ifndef EP_ROUTE_FOLD
+#define EP_ROUTE_FOLD 1   // 0: always the three-phase form
+#endif
+
 namespace ep {
 
 namespace {
 
 constexpr unsigned long long kBarrierTimeoutNs = 2000000000ull;   // a grid barrier gives up after 2 s
+constexpr size_t kRouteFoldSmem = 200 * 1024;   // shared memory the folded routing kernel may take
 
 __device__ __forceinline__ unsigned long long global_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+
+// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all
+// of this thread's copies.
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(sdst))),
+                 "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Grid-wide barrier over a counter that was zero at launch; `target` is
 // gridDim.x times the barrier's ordinal.  False if the wait gave up (after
@@ -114,6 +132,17 @@ __device__ int block_exclusive_scan_E(const int* in, int* out, int E, int* s_war
     return tot;
 }
 
+// Shared memory of the routing kernel without the folded tables, and the
+// (16-byte aligned) offset of the tables after it.
+__host__ __device__ size_t route_smem_bytes(int E, int K, int R, int log2_chunk) {
+    const int C = 1 << log2_chunk;
+    return sizeof(int32_t) * ((size_t)kRouteWarps * E + 3 * (size_t)C * K + R + 3 * (size_t)E + 1 + 40) +
+           (size_t)C * R;
+}
+__host__ __device__ size_t route_table_offset(int E, int K, int R, int log2_chunk) {
+    return (route_smem_bytes(E, K, R, log2_chunk) + 15) & ~size_t(15);
+}
+
 }  // namespace
 
 template <int KT>
@@ -132,6 +161,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     int32_t* s_pad = s_al + E;                        // [E+1] padding prefix
     int32_t* s_misc = s_pad + E + 1;                  // [40]: warp sums, flags
     uint8_t* s_inr = reinterpret_cast<uint8_t*>(s_misc + 40);   // [C][R]
+    // folded routing: [nchunks][E] expert histogram, then [nchunks][R] rank counts
+    int32_t* s_tab = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(smem) +
+                                                 route_table_offset(E, a.K, R, a.log2_chunk));
+    int32_t* s_rtab = s_tab + (size_t)a.nchunks * E;
     int* s_warp = s_misc;
     int* s_flag = s_misc + 32;
     int* s_err = s_misc + 33;
@@ -240,53 +273,83 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         return;
     }
 
-    // ---------------------------------------------------------------- phase 2
-    // column col: [0,E) experts (prefix written in place), [E,E+R) ranks, E+R errors
-    {
-        const int ncol = E + R + 1;
-        for (int col = blockIdx.x * kRouteWarps + warp; col < ncol; col += G * kRouteWarps) {
-            int32_t* tab;
-            int stride, idx;
-            if (col < E) { tab = a.chunk_hist; stride = E; idx = col; }
-            else if (col < E + R) { tab = a.chunk_rcnt; stride = R; idx = col - E; }
-            else { tab = a.chunk_err; stride = 1; idx = 0; }
-            int carry = 0;
-            for (int c0 = 0; c0 < a.nchunks; c0 += 32 * 8) {
-                int v[8];
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const int c = c0 + s * 32 + lane;
-                    v[s] = c < a.nchunks ? __ldcg(tab + (size_t)c * stride + idx) : 0;
-                }
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    int incl = v[s];
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += n;
-                    }
-                    const int c = c0 + s * 32 + lane;
-                    if (col < E && c < a.nchunks) tab[(size_t)c * stride + idx] = carry + incl - v[s];
-                    carry += __shfl_sync(0xffffffffu, incl, 31);
-                }
-            }
-            if (lane == 0) a.col_total[col] = carry;
+    int* s_cnt = wh;   // [E] expert counts (the per-warp table is free now)
+    if (a.fold) {
+        // the tables into shared memory (CTA 0 also takes the rank counts), then
+        // the expert totals; chunk prefixes are summed per chunk below
+        const int n16 = a.nchunks * E / 4;
+        for (int i = tid; i < n16; i += kRouteThreads) cp_async16(s_tab + 4 * i, a.chunk_hist + 4 * i);
+        if (blockIdx.x == 0) {
+            const int r16 = a.nchunks * R / 4;
+            for (int i = tid; i < r16; i += kRouteThreads) cp_async16(s_rtab + 4 * i, a.chunk_rcnt + 4 * i);
         }
-    }
-    if (!grid_barrier(a.barrier, 2u * G, s_flag)) {
-        if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
-        return;
+        cp_async_wait_all();
+        __syncthreads();
+        for (int e = tid; e < E; e += kRouteThreads) {
+            int cnt = 0;
+            for (int c = 0; c < a.nchunks; ++c) cnt += s_tab[(size_t)c * E + e];
+            s_cnt[e] = cnt;
+            s_al[e] = (int)(((int64_t)cnt + a.A - 1) / a.A * a.A);
+        }
+    } else {
+        // ---------------------------------------------------------------- phase 2
+        // column col: [0,E) experts (prefix written in place), [E,E+R) ranks, E+R errors
+        {
+            const int ncol = E + R + 1;
+            for (int col = blockIdx.x * kRouteWarps + warp; col < ncol; col += G * kRouteWarps) {
+                int32_t* tab;
+                int stride, idx;
+                if (col < E) { tab = a.chunk_hist; stride = E; idx = col; }
+                else if (col < E + R) { tab = a.chunk_rcnt; stride = R; idx = col - E; }
+                else { tab = a.chunk_err; stride = 1; idx = 0; }
+                int carry = 0;
+                for (int c0 = 0; c0 < a.nchunks; c0 += 32 * 8) {
+                    int v[8];
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        const int c = c0 + s * 32 + lane;
+                        v[s] = c < a.nchunks ? __ldcg(tab + (size_t)c * stride + idx) : 0;
+                    }
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        int incl = v[s];
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                            if (lane >= o) incl += n;
+                        }
+                        const int c = c0 + s * 32 + lane;
+                        if (col < E && c < a.nchunks) tab[(size_t)c * stride + idx] = carry + incl - v[s];
+                        carry += __shfl_sync(0xffffffffu, incl, 31);
+                    }
+                }
+                if (lane == 0) a.col_total[col] = carry;
+            }
+        }
+        if (!grid_barrier(a.barrier, 2u * G, s_flag)) {
+            if (tid == 0) set_error(a.err_out, EP_ERR_TIMEOUT);
+            return;
+        }
+
+        // the expert counts = the column totals
+        for (int e = tid; e < E; e += kRouteThreads) {
+            const int cnt = __ldcg(a.col_total + e);
+            s_cnt[e] = cnt;
+            s_al[e] = (int)(((int64_t)cnt + a.A - 1) / a.A * a.A);
+        }
     }
 
     // ---------------------------------------------------------------- phase 3
-    int* s_cnt = wh;   // [E] expert counts (the per-warp table is free now)
-    for (int e = tid; e < E; e += kRouteThreads) {
-        const int cnt = __ldcg(a.col_total + e);
-        s_cnt[e] = cnt;
-        s_al[e] = (int)(((int64_t)cnt + a.A - 1) / a.A * a.A);
+    // a bad expert id in any chunk (only CTA 0 reports it)
+    int bad_ids = 0;
+    if (blockIdx.x == 0) {
+        if (a.fold) {
+            for (int c = tid; c < a.nchunks; c += kRouteThreads) bad_ids |= __ldcg(a.chunk_err + c);
+        } else if (tid == 0) {
+            bad_ids = __ldcg(a.col_total + E + R);
+        }
     }
-    __syncthreads();
+    bad_ids = __syncthreads_or(bad_ids);
     const int rows = block_exclusive_scan_E(s_al, s_seg, E, s_warp);
     for (int e = tid; e < E; e += kRouteThreads) s_al[e] -= s_cnt[e];   // padding rows of e
     __syncthreads();
@@ -302,10 +365,18 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
             if (a.num_tokens_per_expert) a.num_tokens_per_expert[e] = cnt;
             if (a.cumulative) a.cumulative[e] += cnt;
         }
-        for (int r = tid; r < R; r += kRouteThreads)
-            if (a.num_tokens_per_rank) a.num_tokens_per_rank[r] = __ldcg(a.col_total + E + r);
+        for (int r = tid; r < R; r += kRouteThreads) {
+            if (!a.num_tokens_per_rank) break;
+            int n = 0;
+            if (a.fold) {
+                for (int c = 0; c < a.nchunks; ++c) n += s_rtab[(size_t)c * R + r];
+            } else {
+                n = __ldcg(a.col_total + E + r);
+            }
+            a.num_tokens_per_rank[r] = n;
+        }
         if (tid == 0) {
-            int status = __ldcg(a.col_total + E + R) ? EP_ERR_BAD_EXPERT_ID : 0;
+            int status = bad_ids ? EP_ERR_BAD_EXPERT_ID : 0;
             if (status == 0 && a.check_capacity && a.ll_M == 0 && (int64_t)rows > a.capacity)
                 status = EP_ERR_CAPACITY;
             if (status) set_error(a.err_out, status);
@@ -321,7 +392,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         const int ne = min(C, a.tokens_per_rank - (c % a.chunks_per_rank) * C) * K;
         const int64_t e0 = (int64_t)t0 * K;
         __syncthreads();
-        if (a.ll_M) {
+        if (a.fold) {
+            // the chunk's prefix: entries of expert e in the chunks before c (from
+            // the source rank's first chunk in the low-latency layout)
+            const int cfirst = a.ll_M ? r_src * a.chunks_per_rank : 0;
+            for (int e = tid; e < E; e += kRouteThreads) {
+                int p = 0;
+                for (int cc = cfirst; cc < c; ++cc) p += s_tab[(size_t)cc * E + e];
+                s_pre[e] = p;
+            }
+        } else if (a.ll_M) {
             // position inside (expert, source rank) = prefix from the rank's first chunk
             const size_t c0 = (size_t)r_src * a.chunks_per_rank;
             for (int e = tid; e < E; e += kRouteThreads)
@@ -395,12 +475,19 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         // per (expert, source rank): (first row of the rank's block << 32) | entries
         for (int i = blockIdx.x * kRouteThreads + tid; i < E * R; i += G * kRouteThreads) {
             const int e = i / R, r = i - e * R;
-            const bool any = a.chunks_per_rank > 0;
-            const int lo = any ? __ldcg(a.chunk_hist + (size_t)r * a.chunks_per_rank * E + e) : 0;
-            const int hi = !any ? 0
-                           : r + 1 < R ? __ldcg(a.chunk_hist + (size_t)(r + 1) * a.chunks_per_rank * E + e)
-                                       : s_cnt[e];
-            if (a.layout_range) a.layout_range[i] = ((int64_t)r * a.ll_M << 32) | (int64_t)(hi - lo);
+            int n = 0;
+            if (a.fold) {
+                for (int c = r * a.chunks_per_rank; c < (r + 1) * a.chunks_per_rank; ++c)
+                    n += s_tab[(size_t)c * E + e];
+            } else {
+                const bool any = a.chunks_per_rank > 0;
+                const int lo = any ? __ldcg(a.chunk_hist + (size_t)r * a.chunks_per_rank * E + e) : 0;
+                const int hi = !any ? 0
+                               : r + 1 < R ? __ldcg(a.chunk_hist + (size_t)(r + 1) * a.chunks_per_rank * E + e)
+                                           : s_cnt[e];
+                n = hi - lo;
+            }
+            if (a.layout_range) a.layout_range[i] = ((int64_t)r * a.ll_M << 32) | (int64_t)n;
         }
         return;   // no padding rows in the fixed-capacity layout
     }
@@ -421,17 +508,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     }
 }
 
-size_t route_smem_bytes(int E, int K, int R, int log2_chunk) {
-    const int C = 1 << log2_chunk;
-    return sizeof(int32_t) * ((size_t)kRouteWarps * E + 3 * (size_t)C * K + R + 3 * (size_t)E + 1 + 40) +
-           (size_t)C * R;
-}
+
+
 
 namespace {
 
 template <int KT>
 cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
-    const size_t smem = route_smem_bytes(a.E, a.K, a.R, a.log2_chunk);
+    const size_t smem = a.fold ? route_table_offset(a.E, a.K, a.R, a.log2_chunk) +
+                                     sizeof(int32_t) * (size_t)a.nchunks * (a.E + a.R)
+                               : route_smem_bytes(a.E, a.K, a.R, a.log2_chunk);
     cudaError_t e = cudaFuncSetAttribute(k_route<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -455,9 +541,18 @@ cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
-    cudaError_t e = cudaMemsetAsync(a.barrier, 0, sizeof(unsigned), st);
+cudaError_t launch_route(const RouteArgs& args, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(args.barrier, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return e;
+    RouteArgs a = args;
+    // fold the column phase when both tables fit in shared memory with the rest
+    const size_t tables = sizeof(int32_t) * (size_t)a.nchunks * (a.E + a.R);
+    // (whole 16-byte pieces at 16-byte aligned addresses), and every chunk has
+    // its own CTA at one CTA per SM
+    a.fold = EP_ROUTE_FOLD && ((size_t)a.nchunks * a.E) % 4 == 0 && ((size_t)a.nchunks * a.R) % 4 == 0 &&
+             (reinterpret_cast<uintptr_t>(a.chunk_hist) & 15u) == 0 &&
+             (reinterpret_cast<uintptr_t>(a.chunk_rcnt) & 15u) == 0 && a.nchunks <= device_sm_count() &&
+             route_table_offset(a.E, a.K, a.R, a.log2_chunk) + tables <= kRouteFoldSmem;
     switch (a.vector_ok ? a.K : 0) {
         case 4: return launch_route_k<4>(a, st);
         case 8: return launch_route_k<8>(a, st);
