@@ -142,6 +142,11 @@ __host__ __device__ size_t route_smem_bytes(int E, int K, int R, int log2_chunk)
 __host__ __device__ size_t route_table_offset(int E, int K, int R, int log2_chunk) {
     return (route_smem_bytes(E, K, R, log2_chunk) + 15) & ~size_t(15);
 }
+// Folded tables: [nchunks][E] + [nchunks][R] int32, then [2][threads] int4
+// partial column sums.
+size_t route_fold_bytes(const RouteArgs& a) {
+    return sizeof(int32_t) * (size_t)a.nchunks * (a.E + a.R) + 2 * sizeof(int4) * kRouteThreads;
+}
 
 }  // namespace
 
@@ -165,6 +170,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     int32_t* s_tab = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(smem) +
                                                  route_table_offset(E, a.K, R, a.log2_chunk));
     int32_t* s_rtab = s_tab + (size_t)a.nchunks * E;
+    int32_t* s_fpre = wh + E;  // [E] folded: this chunk's prefix (wh[0, E) holds the expert counts)
     int* s_warp = s_misc;
     int* s_flag = s_misc + 32;
     int* s_err = s_misc + 33;
@@ -188,19 +194,34 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         const int nt = min(C, a.tokens_per_rank - (c % a.chunks_per_rank) * C);
         const int ne = nt * K;
         const int64_t e0 = (int64_t)t0 * K;
-        for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wh[i] = 0;
-        for (int i = tid; i < R; i += kRouteThreads) s_rcnt[i] = 0;
-        for (int i = tid; i < nt * R; i += kRouteThreads) s_inr[i] = 0;
-        if (tid == 0) *s_err = 0;
-        // this warp's entries (and, for dispatch, the chunk's weights), all loads issued up front
+        // this warp's entries (and, for dispatch, the chunk's weights): every
+        // load is issued first, the shared tables are cleared while they fly
         int64_t ld[kMaxBatches];
 #pragma unroll
         for (int b = 0; b < kMaxBatches; ++b) {
             const int i = warp * per_warp + b * 32 + lane;
             ld[b] = (b < nb && i < ne) ? a.topk_idx[e0 + i] : -1;
         }
-        if (a.assign)
-            for (int i = tid; i < ne; i += kRouteThreads) s_w[i] = a.topk_weights[e0 + i];
+        constexpr int kW = kMaxChunkEntries / kRouteThreads;   // weights per thread
+        float wv[kW];
+        if (a.assign) {
+#pragma unroll
+            for (int j = 0; j < kW; ++j) {
+                const int i = tid + j * kRouteThreads;
+                wv[j] = i < ne ? a.topk_weights[e0 + i] : 0.0f;
+            }
+        }
+        for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wh[i] = 0;
+        for (int i = tid; i < R; i += kRouteThreads) s_rcnt[i] = 0;
+        for (int i = tid; i < nt * R; i += kRouteThreads) s_inr[i] = 0;
+        if (tid == 0) *s_err = 0;
+        if (a.assign) {
+#pragma unroll
+            for (int j = 0; j < kW; ++j) {
+                const int i = tid + j * kRouteThreads;
+                if (i < ne) s_w[i] = wv[j];
+            }
+        }
         __syncthreads();
         int my_e[kMaxBatches], my_r[kMaxBatches];
 #pragma unroll
@@ -285,11 +306,37 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         }
         cp_async_wait_all();
         __syncthreads();
+        // one pass over the table: thread (q, g) sums columns 4q..4q+3 over
+        // rows g, g + RG, ... into the total and into this CTA's chunk prefix
+        // (rows [cfirst, c): from the source rank's first chunk in the
+        // low-latency layout); the RG partial sums of a column meet in s_part
+        const int c = blockIdx.x;   // folded: one chunk per CTA
+        const int cfirst = a.ll_M ? (c / a.chunks_per_rank) * a.chunks_per_rank : 0;
+        const int QE = E / 4, RG = kRouteThreads / QE;
+        const int q = tid % QE, g = tid / QE;
+        int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+        if (g < RG) {
+            const int4* t4 = reinterpret_cast<const int4*>(s_tab);
+            for (int r = g; r < a.nchunks; r += RG) {
+                const int4 v = t4[(size_t)r * QE + q];
+                tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+                if (r >= cfirst && r < c) { pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w; }
+            }
+        }
+        int4* s_part = reinterpret_cast<int4*>(s_rtab + (size_t)a.nchunks * R);   // [2][kRouteThreads]
+        s_part[tid] = tot;
+        s_part[kRouteThreads + tid] = pre;
+        __syncthreads();
+        const int* pt = reinterpret_cast<const int*>(s_part);
         for (int e = tid; e < E; e += kRouteThreads) {
-            int cnt = 0;
-            for (int c = 0; c < a.nchunks; ++c) cnt += s_tab[(size_t)c * E + e];
+            int cnt = 0, p = 0;
+            for (int j = 0; j < RG; ++j) {
+                cnt += pt[j * E + e];
+                p += pt[4 * kRouteThreads + j * E + e];
+            }
             s_cnt[e] = cnt;
             s_al[e] = (int)(((int64_t)cnt + a.A - 1) / a.A * a.A);
+            s_fpre[e] = p;
         }
     } else {
         // ---------------------------------------------------------------- phase 2
@@ -393,14 +440,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         const int64_t e0 = (int64_t)t0 * K;
         __syncthreads();
         if (a.fold) {
-            // the chunk's prefix: entries of expert e in the chunks before c (from
-            // the source rank's first chunk in the low-latency layout)
-            const int cfirst = a.ll_M ? r_src * a.chunks_per_rank : 0;
-            for (int e = tid; e < E; e += kRouteThreads) {
-                int p = 0;
-                for (int cc = cfirst; cc < c; ++cc) p += s_tab[(size_t)cc * E + e];
-                s_pre[e] = p;
-            }
+            // the chunk's prefix, summed with the totals
+            for (int e = tid; e < E; e += kRouteThreads) s_pre[e] = s_fpre[e];
         } else if (a.ll_M) {
             // position inside (expert, source rank) = prefix from the rank's first chunk
             const size_t c0 = (size_t)r_src * a.chunks_per_rank;
@@ -515,8 +556,7 @@ namespace {
 
 template <int KT>
 cudaError_t launch_route_k(const RouteArgs& a, cudaStream_t st) {
-    const size_t smem = a.fold ? route_table_offset(a.E, a.K, a.R, a.log2_chunk) +
-                                     sizeof(int32_t) * (size_t)a.nchunks * (a.E + a.R)
+    const size_t smem = a.fold ? route_table_offset(a.E, a.K, a.R, a.log2_chunk) + route_fold_bytes(a)
                                : route_smem_bytes(a.E, a.K, a.R, a.log2_chunk);
     cudaError_t e = cudaFuncSetAttribute(k_route<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -546,13 +586,12 @@ cudaError_t launch_route(const RouteArgs& args, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     RouteArgs a = args;
     // fold the column phase when both tables fit in shared memory with the rest
-    const size_t tables = sizeof(int32_t) * (size_t)a.nchunks * (a.E + a.R);
-    // (whole 16-byte pieces at 16-byte aligned addresses), and every chunk has
-    // its own CTA at one CTA per SM
-    a.fold = EP_ROUTE_FOLD && ((size_t)a.nchunks * a.E) % 4 == 0 && ((size_t)a.nchunks * a.R) % 4 == 0 &&
+    // (whole 16-byte pieces at 16-byte aligned addresses, rows of whole
+    // 16-byte column groups), and every chunk has its own CTA at one CTA per SM
+    a.fold = EP_ROUTE_FOLD && a.E % 4 == 0 && ((size_t)a.nchunks * a.R) % 4 == 0 &&
              (reinterpret_cast<uintptr_t>(a.chunk_hist) & 15u) == 0 &&
              (reinterpret_cast<uintptr_t>(a.chunk_rcnt) & 15u) == 0 && a.nchunks <= device_sm_count() &&
-             route_table_offset(a.E, a.K, a.R, a.log2_chunk) + tables <= kRouteFoldSmem;
+             route_table_offset(a.E, a.K, a.R, a.log2_chunk) + route_fold_bytes(a) <= kRouteFoldSmem;
     switch (a.vector_ok ? a.K : 0) {
         case 4: return launch_route_k<4>(a, st);
         case 8: return launch_route_k<8>(a, st);
