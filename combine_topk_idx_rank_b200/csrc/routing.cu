@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
         // (rows [cfirst, c): from the source rank's first chunk in the
         // low-latency layout); the RG partial sums of a column meet in s_part
         const int c = blockIdx.x;   // folded: one chunk per CTA
-        const int cfirst = a.ll_M ? (c / a.chunks_per_rank) * a.chunks_per_rank : 0;
+        const int cfirst = a.ll_M && a.chunks_per_rank > 0 ? (c / a.chunks_per_rank) * a.chunks_per_rank : 0;
         const int QE = E / 4, RG = kRouteThreads / QE;
         const int q = tid % QE, g = tid / QE;
         int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
