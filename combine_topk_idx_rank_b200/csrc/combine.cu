@@ -24,6 +24,25 @@
 
 namespace ep {
 
+// Packed fp32 pairs (sm_100): each half is the same correctly rounded
+// operation as its scalar form, so results are bit-identical.
+//   (r0, r1) = (a0 * b, a1 * b)          (d0, d1) = (w * a0 + d0, w * a1 + d1)
+__device__ __forceinline__ void mul2_rn(float& r0, float& r1, float a0, float a1, float b) {
+    uint64_t x, y, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(b));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float w, float a0, float a1) {
+    uint64_t ww, x, d;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(ww) : "f"(w));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(ww), "l"(x), "l"(d));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 // Eight codes -> decode(code) * scale (fp32 product).  YQ 1 = FP8 e4m3
 // (decoded exactly through fp16), 2 = int8.
 template <int YQ>
@@ -46,7 +65,7 @@ __device__ __forceinline__ void dequant8(uint2 c, float s, float (&v)[8]) {
         }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], s);
+    for (int i = 0; i < 8; i += 2) mul2_rn(v[i], v[i + 1], v[i], v[i + 1], s);
 }
 
 template <int KMAX, int VPT>
@@ -209,9 +228,9 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine_q(Combin
                     dequant8<YQ>(make_uint2(q[j].x, q[j].y), sc[j], lo);
                     dequant8<YQ>(make_uint2(q[j].z, q[j].w), sc[j], hi);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        acc[i] = __fmaf_rn(w, lo[i], acc[i]);
-                        acc[8 + i] = __fmaf_rn(w, hi[i], acc[8 + i]);
+                    for (int i = 0; i < 8; i += 2) {
+                        fma2_rn(acc[i], acc[i + 1], w, lo[i], lo[i + 1]);
+                        fma2_rn(acc[8 + i], acc[8 + i + 1], w, hi[i], hi[i + 1]);
                     }
                 }
             }
