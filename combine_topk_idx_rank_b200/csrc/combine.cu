@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256, EP_COMBINE_MIN_BLOCKS) k_combine(CombineA
                         y[0] = bf16lo(b.x); y[1] = bf16hi(b.x); y[2] = bf16lo(b.y); y[3] = bf16hi(b.y);
                         y[4] = bf16lo(b.z); y[5] = bf16hi(b.z); y[6] = bf16lo(b.w); y[7] = bf16hi(b.w);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, y[i], acc[i]);
+                        for (int i = 0; i < 8; i += 2) fma2_rn(acc[i], acc[i + 1], w, y[i], y[i + 1]);
                     }
                 }
                 if (v < V) {
