@@ -148,9 +148,6 @@ __device__ __forceinline__ void load_slots(const PackArgs& a, int t, int* s_slot
 // 0..K-1 fetch the unit's destination rows one iteration ahead of use.
 template <int S>
 __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
-    grid_dependency_wait();
-    grid_launch_dependents();
-    if (routing_gave_up(a)) return;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* stage = smem;
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + (size_t)S * chunk_bytes);
@@ -170,8 +167,6 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         for (int s = 0; s < S; ++s) mbar_init(&mbar[s], 1);
         fence_mbar_init();
     }
-    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
-    __syncwarp();
 
     auto unit = [&](int j, int& t, int& c) {
         const int u = (int)blockIdx.x + j * (int)gridDim.x;
@@ -187,12 +182,33 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         bulk_load(stage + (size_t)(j % S) * chunk_bytes, xb + (int64_t)t * row_bytes + off, bytes, bar);
     };
 
-    // prologue: units 0 .. S-2
+    // prologue: units 0 .. S-2.  With routing just ahead on the stream (x
+    // complete before it started) their x chunks are requested before the
+    // wait for the routing results, while routing runs
     const int pro = min(S - 1, n_mine);
+    const bool early = a.early_x != 0;
+    if (early && lane == 0) {
+        for (int j = 0; j < pro; ++j) {
+            int t, c;
+            unit(j, t, c);
+            issue_load(j, t, c);
+        }
+    }
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (routing_gave_up(a)) {
+        // the chunks requested early land before the CTA releases its smem
+        if (early && lane == 0)
+            for (int j = 0; j < pro; ++j) mbar_wait(&mbar[j % S], (uint32_t)((j / S) & 1));
+        __syncwarp();
+        return;
+    }
+    const int n_pad = a.do_pad ? build_pad_map(a, s_pad_base, s_pad_start, s_warp) : 0;
+    __syncwarp();
     for (int j = 0; j < pro; ++j) {
         int t, c;
         unit(j, t, c);
-        if (lane == 0) issue_load(j, t, c);
+        if (!early && lane == 0) issue_load(j, t, c);
         if (lane < K) sslot[(j % S) * kMaxTopk + lane] = checked_row(a, a.dst_slot[(int64_t)t * K + lane]);
     }
     __syncwarp();

@@ -54,12 +54,13 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // Grid-wide barrier over a counter that was zero at launch; `target` is
 // gridDim.x times the barrier's ordinal.  False if the wait gave up (after
-// kBarrierTimeoutNs of the global timer).
+// kBarrierTimeoutNs of the global timer).  Thread 0 arrives with a release
+// reduction (after the block barrier it covers the whole CTA's writes) and
+// polls with acquire loads; the closing block barrier hands the acquire on.
 __device__ bool grid_barrier(unsigned* counter, unsigned target, int* s_flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(counter, 1u);
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
         int ok = 1;
         const unsigned long long t0 = global_ns();
         for (;;) {
@@ -70,9 +71,8 @@ __device__ bool grid_barrier(unsigned* counter, unsigned target, int* s_flag) {
                 ok = 0;
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
         }
-        __threadfence();
         *s_flag = ok;
     }
     __syncthreads();
@@ -399,8 +399,11 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteArgs a) {
     bad_ids = __syncthreads_or(bad_ids);
     const int rows = block_exclusive_scan_E(s_al, s_seg, E, s_warp);
     for (int e = tid; e < E; e += kRouteThreads) s_al[e] -= s_cnt[e];   // padding rows of e
-    __syncthreads();
-    const int pads = block_exclusive_scan_E(s_al, s_pad, E, s_warp);
+    int pads = 0;
+    if (a.A > 1) {   // with expert_alignment 1 there are no padding rows to number
+        __syncthreads();
+        pads = block_exclusive_scan_E(s_al, s_pad, E, s_warp);
+    }
     if (tid == 0) s_pad[E] = pads;
     __syncthreads();
 
