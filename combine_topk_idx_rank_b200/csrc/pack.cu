@@ -18,7 +18,8 @@
 // ring in shared memory; lane 0 streams row chunks in with cp.async.bulk
 // (completion on an mbarrier) and, once a chunk has landed, issues one
 // cp.async.bulk store per destination row from the same shared-memory stage.
-// No register ever holds row data, and no multicast is used.
+// No register ever holds row data; every bulk copy fills or drains this
+// CTA's own shared memory.
 // Quantised rows are computed by threads from 16-byte vector loads and
 // written with 16-byte vector stores.
 #include <cuda_bf16.h>

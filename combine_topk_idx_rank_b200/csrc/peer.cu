@@ -18,7 +18,7 @@
 // scales, quantised once) and each entry's recv_topk_idx / weights / metadata
 // row straight into the receiver's layout; k_combine_peer loads each token's
 // rows from the receivers' expert outputs and reduces them in k order.  Plain
-// peer loads and stores only: no multicast, no waits on other GPUs (the
+// peer loads and stores only, and no waits on other GPUs (the
 // caller's collectives order the steps).
 #include "ep_internal.cuh"
 #include "quant.cuh"

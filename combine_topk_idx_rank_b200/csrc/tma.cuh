@@ -1,5 +1,6 @@
 // TMA bulk-copy and mbarrier primitives (inline PTX for sm_100a) shared by the
-// pack and routing kernels.  No multicast form is used anywhere.
+// pack and routing kernels.  Each copy moves data between global memory and
+// the issuing CTA's own shared memory.
 #pragma once
 
 #include <stdint.h>

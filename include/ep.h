@@ -359,7 +359,7 @@ ep_status_t ep_write_padding_rows(const int32_t* psum, const int32_t* counts, in
  * Peer pointer tables are device arrays of G pointers (entry g' = that
  * buffer on GPU g', mapped into this process; entry g = this GPU's own).
  * Nothing here waits on another GPU: the caller's collectives order the
- * steps.  No TMA or bulk load with cluster multicast is used.
+ * steps.  Peer memory is reached with plain loads and stores only.
  */
 
 /* Routing only (steps 1): ep_dispatch's handle, recv_topk_idx,
