@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(32) k_pack_bulk(PackArgs a, int chunk_bytes) {
         const int s = i % S;
         // slots fetched last iteration belong to unit i + S - 2
         if (i >= 1 && i + S - 2 < n_mine && lane < K) sslot[((i + S - 2) % S) * kMaxTopk + lane] = checked_row(a, pending);
-        // lane 0 waits for the stage; the verdict is broadcast so the warp stays converged
+        // lane 0 waits for the stage; the outcome is broadcast so the warp stays converged
         int landed = lane == 0 ? (int)mbar_wait(&mbar[s], (uint32_t)((i / S) & 1)) : 0;
         landed = __shfl_sync(0xffffffffu, landed, 0);
         if (!landed) {
