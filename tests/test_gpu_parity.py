@@ -458,3 +458,68 @@ def test_e2m1_conversion_over_bf16(cuda_device):
     assert np.all(ref_s == 127)
     assert np.array_equal(recv_x.cpu().numpy(), ref_x)
     assert np.array_equal(recv_scales.cpu().numpy(), ref_s)
+
+
+def _offset_workspace(nbytes, off, dev):
+    """A workspace of nbytes starting `off` bytes into a larger allocation."""
+    big = torch.empty((nbytes + 256,), dtype=torch.uint8, device=dev)
+    return big[off:off + nbytes]
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "qwen3"])
+def test_routing_forms_agree(name, cuda_device):
+    """The folded routing form (the per-chunk tables copied whole into shared
+    memory after one grid barrier) and the three-phase form (column prefixes
+    in the workspace, a second barrier) give the same bits.  The folded form
+    needs its workspace tables 16-byte aligned, so a workspace that starts 4
+    bytes into an allocation takes the three-phase form on the same shape."""
+    dev = cuda_device
+    cfg = _small(name)
+    T, H, K, E, R, A = (cfg.num_tokens, cfg.hidden, cfg.num_topk, cfg.num_experts, cfg.num_ranks,
+                        cfg.expert_alignment)
+    q = None if cfg.quant == "none" else cfg.quant
+    wl = make_workload(cfg, 3)
+    ref = oracle.dispatch(wl.x, wl.topk_idx, wl.topk_weights, E, R, A, cfg.quant, cfg.quant_size, cfg.round_scale,
+                          cfg.num_rounds)
+    ref_lay = oracle.layout(wl.topk_idx, E, R)
+    got = []
+    for off in (0, 4):
+        bufs = ep.alloc_dispatch_buffers(T, H, K, E, R, A, q, cfg.quant_size, cfg.num_rounds, device=dev)
+        bufs.workspace = _offset_workspace(bufs.workspace.numel(), off, dev)
+        (recv_x, recv_scales, rti, rtw, h), lay, _ = gpu_dispatch(cfg, wl, dev, buffers=bufs)
+        assert_layout_equal(lay, ref_lay)
+        assert_slots_equal(h, rti, rtw, ref)
+        assert_rows_equal(cfg, recv_x, recv_scales, ref["recv_x"], ref["recv_scales"])
+        n = h.num_recv_rows
+        got.append([u8(recv_x[:n]), h.dst_buffer_slot_idx.cpu().numpy(), h.recv_src_metadata[:n].cpu().numpy()])
+    for a, b in zip(*got):
+        assert np.array_equal(a, b)
+
+
+def test_low_latency_routing_forms_agree(cuda_device):
+    """The same for the low-latency layout, whose positions count from each
+    source rank's first chunk."""
+    dev = cuda_device
+    cfg = CONFIGS["decode"].scaled(num_tokens=16 * 40, hidden=1024)
+    wl = make_workload(cfg, 4)
+    T, K, E, R, M = cfg.num_tokens, cfg.num_topk, cfg.num_experts, cfg.num_ranks, 48
+    ref = oracle.ll_slots(wl.topk_idx, wl.topk_weights, E, R, M)
+    x, ti, tw = to_dev(wl, dev)
+    got = []
+    for off in (0, 4):
+        ws = _offset_workspace(ep.workspace_bytes(T, K, E, R), off, dev)
+        recv_x, recv_scales, count, layout_range, h = ep.ep_dispatch_low_latency(
+            x, ti, tw, M, E, R, "fp8", quant_size=128, workspace=ws)
+        torch.cuda.synchronize()
+        assert h.read_error() == ep.EP_OK
+        assert np.array_equal(h.dst_buffer_slot_idx.cpu().numpy(), ref["dst_buffer_slot_idx"])
+        assert np.array_equal(count.cpu().numpy(), ref["recv_count"])
+        assert np.array_equal(layout_range.cpu().numpy(), ref["layout_range"])
+        # the rows that received an entry (the others of the fixed-capacity layout are never written)
+        dst = ref["dst_buffer_slot_idx"]
+        used = np.unique(dst[dst >= 0])
+        rows = E * R * M
+        got.append([u8(recv_x).reshape(rows, -1)[used],
+                    recv_scales.reshape(rows, -1).cpu().numpy().view(np.uint32)[used]])
+    for a, b in zip(*got):
+        assert np.array_equal(a, b)
